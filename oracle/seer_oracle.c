@@ -1,0 +1,417 @@
+/*
+ * seer_oracle.c — plain, slow, fp64 CPU reference for the SeerAttention
+ * prefill hot path (AttnGate scores, block mask, compaction, block-sparse
+ * causal attention, and the Figure 8 max-pooled attention map).
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing in the product path may link, load or
+ * call this file: only the tests, the smoke check and the CPU-baseline leg of
+ * the benchmark use it.  It shares no code, header, table or helper with the
+ * CUDA library.  Every loop follows the definition it cites; there is no
+ * tiling, fusion or reordering beyond the definition.  Floating point is fp64
+ * throughout; bf16 inputs are widened exactly (bf16 -> fp32 -> fp64).
+ *
+ * Sources (web pages about SeerAttention):
+ *  [GATE]  "SeerAttention: Learning Intrinsic Sparse Attention in Your LLMs",
+ *          rebuttal, Weakness 3 (pooling along the sequence axis, shapes
+ *          [Batch, Head, Seq/Block, Dim], pooling before the linear layer),
+ *          Question 1 on pooling ("Q prefers avg"), Q1 on AttnGate's RoPE
+ *          (block RoPE on non-RoPE'd pooled Q/K), Weakness 2 (the gate is
+ *          "similar to self-attention without the multiply with V"; per-row
+ *          TopK; [Seq/Block, TopK] index tensor).
+ *  [CARD]  "SeerAttention-Llama-3.1-8B-AttnGates" model card: masks come from
+ *          threshold/TopK on the gate's soft scores and drive a block-sparse
+ *          FlashAttention kernel.
+ *  [INF]   same rebuttal, Weakness 5: inference kernel pseudocode (per query
+ *          block, loop over the selected key blocks only, online softmax).
+ *  [FIG8]  "SeerAttention: Self-distilled Attention Gating for Efficient
+ *          Long-context Prefilling", Figure 8: FlashAttention with a max-pooled
+ *          attention map (store the block row max r_ij, then
+ *          a_ij = exp(r_ij - m_i) / l_i and A_ij = colmax(a_ij)).
+ *  [SEC4]  same page, Sec. 4: block size B = 64 for gate and kernel.
+ *
+ * Readings taken where the pages are silent (each is listed in the design
+ * notes): K is average-pooled like Q; the gate projection is per head with no
+ * bias; block RoPE uses position = block index, half-split (rotate-half)
+ * pairs and base theta; the gate softmax is causal over key blocks j <= i with
+ * scale 1/sqrt(d_gate); attention scale defaults to 1/sqrt(d); queries and
+ * keys share positions starting at 0 (top-left causal); the threshold test is
+ * strict (>); forced blocks (first, diagonal) count toward TopK's k; TopK ties
+ * go to the lower block index.
+ *
+ * Parity pins: every function here is checked by the CPU tests against closed
+ * forms, invariants and brute force (see the tests that import oracle/).
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#define SEER_ORACLE_BLOCK 64 /* [SEC4]: block size fixed at 64 */
+
+static double bf16_to_f64(uint16_t bits)
+{
+    uint32_t u = ((uint32_t)bits) << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return (double)f;
+}
+
+/* ---------------------------------------------------------------------------
+ * a1 [GATE Weakness 3]: average pooling along the sequence axis.
+ * x: bf16 [B, H, S, d]  ->  out: f64 [B, H, S/64, d]
+ * out[b,h,i,c] = (1/64) * sum_{t<64} x[b,h,64 i + t, c]
+ * ------------------------------------------------------------------------- */
+void oracle_pool_avg(const uint16_t *x, int B, int H, int S, int d, double *out)
+{
+    const int nb = S / SEER_ORACLE_BLOCK;
+    const long long units = (long long)B * H * nb;
+#pragma omp parallel for schedule(static)
+    for (long long u = 0; u < units; ++u) {
+        const long long bh = u / nb;
+        const int i = (int)(u % nb);
+        const uint16_t *base = x + (bh * S + (long long)i * SEER_ORACLE_BLOCK) * d;
+        double *o = out + u * d;
+        for (int c = 0; c < d; ++c) {
+            double s = 0.0;
+            for (int t = 0; t < SEER_ORACLE_BLOCK; ++t)
+                s += bf16_to_f64(base[(long long)t * d + c]);
+            o[c] = s / SEER_ORACLE_BLOCK;
+        }
+    }
+}
+
+/* ---------------------------------------------------------------------------
+ * Block RoPE [GATE Q1 on AttnGate's RoPE]: rotate-half pairs (t, t + dg/2)
+ * by angle p * theta^(-2t/dg), p = block index.  In place on one vector.
+ * ------------------------------------------------------------------------- */
+void oracle_block_rope(double *x, int dg, int p, double theta)
+{
+    const int half = dg / 2;
+    for (int t = 0; t < half; ++t) {
+        const double ang = (double)p * pow(theta, -2.0 * (double)t / (double)dg);
+        const double c = cos(ang), s = sin(ang);
+        const double x0 = x[t], x1 = x[t + half];
+        x[t] = x0 * c - x1 * s;
+        x[t + half] = x1 * c + x0 * s;
+    }
+}
+
+/* ---------------------------------------------------------------------------
+ * a2 [GATE Weakness 3: pooling happens before the linear layer]:
+ * out[b,h,i,:] = RoPE_i( xp[b,h,i,:] @ W[h] ),  W[h] bf16 [d, dg] row-major
+ * at w + h * w_head_stride (stride in elements; 0 = one shared matrix).
+ * ------------------------------------------------------------------------- */
+void oracle_project_rope(const double *xp, int B, int H, int nb, int d,
+                         const uint16_t *w, long long w_head_stride, int dg,
+                         double theta, double *out)
+{
+    const long long units = (long long)B * H * nb;
+#pragma omp parallel for schedule(static)
+    for (long long u = 0; u < units; ++u) {
+        const int h = (int)((u / nb) % H);
+        const int i = (int)(u % nb);
+        const double *xv = xp + u * d;
+        const uint16_t *wh = w + (long long)h * w_head_stride;
+        double *o = out + u * dg;
+        for (int e = 0; e < dg; ++e) {
+            double s = 0.0;
+            for (int c = 0; c < d; ++c)
+                s += xv[c] * bf16_to_f64(wh[(long long)c * dg + e]);
+            o[e] = s;
+        }
+        oracle_block_rope(o, dg, i, theta);
+    }
+}
+
+/* ---------------------------------------------------------------------------
+ * a3 [GATE Weakness 2: "similar to self-attention without the multiply with
+ * V"; Question 2: the gate output rows sum to 1]:
+ * G[b,h,i,j] = softmax_{j<=i}( qt[b,h,i] . kt[b,h/g,j] / sqrt(dg) ), 0 for j>i.
+ * Full chain: pool Q and K, project + block RoPE, causal block softmax.
+ * scores: f64 [B, Hq, nb, nb].
+ * ------------------------------------------------------------------------- */
+void oracle_block_softmax(const double *qt, const double *kt, int B, int Hq,
+                          int Hkv, int nb, int dg, double *scores)
+{
+    const int g = Hq / Hkv;
+    const long long units = (long long)B * Hq * nb;
+    const double scale = 1.0 / sqrt((double)dg);
+#pragma omp parallel for schedule(dynamic, 16)
+    for (long long u = 0; u < units; ++u) {
+        const int b = (int)(u / ((long long)Hq * nb));
+        const int h = (int)((u / nb) % Hq);
+        const int i = (int)(u % nb);
+        const double *qv = qt + u * dg;
+        const double *kbase = kt + ((long long)b * Hkv + h / g) * nb * dg;
+        double *row = scores + u * nb;
+        double m = -INFINITY;
+        for (int j = 0; j <= i; ++j) {
+            double s = 0.0;
+            for (int e = 0; e < dg; ++e)
+                s += qv[e] * kbase[(long long)j * dg + e];
+            row[j] = s * scale;
+            if (row[j] > m)
+                m = row[j];
+        }
+        double l = 0.0;
+        for (int j = 0; j <= i; ++j) {
+            row[j] = exp(row[j] - m);
+            l += row[j];
+        }
+        for (int j = 0; j <= i; ++j)
+            row[j] /= l;
+        for (int j = i + 1; j < nb; ++j)
+            row[j] = 0.0;
+    }
+}
+
+void oracle_gate_scores(const uint16_t *q, const uint16_t *k, int B, int Hq,
+                        int Hkv, int S, int d, const uint16_t *wq,
+                        long long wq_head_stride, const uint16_t *wk,
+                        long long wk_head_stride, int dg, double theta,
+                        double *scores)
+{
+    const int nb = S / SEER_ORACLE_BLOCK;
+    double *qp = (double *)malloc(sizeof(double) * (size_t)B * Hq * nb * d);
+    double *kp = (double *)malloc(sizeof(double) * (size_t)B * Hkv * nb * d);
+    double *qt = (double *)malloc(sizeof(double) * (size_t)B * Hq * nb * dg);
+    double *kt = (double *)malloc(sizeof(double) * (size_t)B * Hkv * nb * dg);
+    oracle_pool_avg(q, B, Hq, S, d, qp);
+    oracle_pool_avg(k, B, Hkv, S, d, kp);
+    oracle_project_rope(qp, B, Hq, nb, d, wq, wq_head_stride, dg, theta, qt);
+    oracle_project_rope(kp, B, Hkv, nb, d, wk, wk_head_stride, dg, theta, kt);
+    oracle_block_softmax(qt, kt, B, Hq, Hkv, nb, dg, scores);
+    free(qp);
+    free(kp);
+    free(qt);
+    free(kt);
+}
+
+/* ---------------------------------------------------------------------------
+ * a4 [CARD: threshold/TopK on the soft scores gives a binary block mask;
+ * GATE Weakness 2: TopK is per row, not global].
+ * scores: f32 [B, Hq, nb, nb] (the values the mask is decided from; the
+ * comparison itself is done in f64 on the widened values).
+ * Threshold (mode 0): keep j <= i with score > threshold.
+ * TopK (mode 1): keep exactly k_i = clamp(k_row[i], |F_i|, i+1) blocks of row
+ * i: first the forced set F_i, then the largest remaining scores, ties to the
+ * lower j.  In both modes block 0 (force_first) and block i (force_diag) are
+ * kept.  mask: u8 [B, Hq, nb, nb], 0 for j > i.
+ * ------------------------------------------------------------------------- */
+int oracle_topk_count(double density, int i, int n_forced)
+{
+    /* k_i = ceil(density * (i+1)) clamped to [n_forced, i+1]. */
+    double want = ceil(density * (double)(i + 1));
+    int k = (want > (double)(i + 1)) ? (i + 1) : (int)want;
+    if (k < n_forced)
+        k = n_forced;
+    if (k > i + 1)
+        k = i + 1;
+    return k;
+}
+
+void oracle_block_mask(const float *scores, int B, int Hq, int nb, int mode,
+                       float threshold, const int32_t *k_row, int force_first,
+                       int force_diag, uint8_t *mask)
+{
+    const long long units = (long long)B * Hq * nb;
+#pragma omp parallel for schedule(dynamic, 16)
+    for (long long u = 0; u < units; ++u) {
+        const int i = (int)(u % nb);
+        const float *row = scores + u * nb;
+        uint8_t *mrow = mask + u * nb;
+        memset(mrow, 0, (size_t)nb);
+        int n_forced = 0;
+        if (force_first) {
+            mrow[0] = 1;
+            n_forced = 1;
+        }
+        if (force_diag && !mrow[i]) {
+            mrow[i] = 1;
+            n_forced += 1;
+        }
+        if (mode == 0) {
+            for (int j = 0; j <= i; ++j)
+                if ((double)row[j] > (double)threshold)
+                    mrow[j] = 1;
+        } else {
+            int k = k_row[i];
+            if (k < n_forced)
+                k = n_forced;
+            if (k > i + 1)
+                k = i + 1;
+            /* Selection by repeated arg-max over the not-yet-chosen blocks:
+             * the largest score wins, the lower j wins a tie. */
+            for (int taken = n_forced; taken < k; ++taken) {
+                int best = -1;
+                for (int j = 0; j <= i; ++j) {
+                    if (mrow[j])
+                        continue;
+                    if (best < 0 || (double)row[j] > (double)row[best])
+                        best = j;
+                }
+                mrow[best] = 1;
+            }
+        }
+    }
+}
+
+/* ---------------------------------------------------------------------------
+ * a5 [INF: "for j from 1 to TopK ... sparse block index"; GATE Weakness 2:
+ * [Seq/Block, TopK] index tensor]: per (b, h, i) the ascending list of active
+ * key blocks j <= i.  Lists are stored causal-packed: row i of head (b, h)
+ * starts at (b*Hq + h) * nb(nb+1)/2 + i(i+1)/2 and has room for i+1 entries;
+ * unused entries are left untouched.  counts: i32 [B, Hq, nb].
+ * ------------------------------------------------------------------------- */
+void oracle_compact(const uint8_t *mask, int B, int Hq, int nb, int32_t *lists,
+                    int32_t *counts)
+{
+    const long long tri = (long long)nb * (nb + 1) / 2;
+    const long long units = (long long)B * Hq * nb;
+    for (long long u = 0; u < units; ++u) {
+        const long long bh = u / nb;
+        const int i = (int)(u % nb);
+        const uint8_t *mrow = mask + u * nb;
+        int32_t *out = lists + bh * tri + (long long)i * (i + 1) / 2;
+        int n = 0;
+        for (int j = 0; j <= i; ++j)
+            if (mrow[j])
+                out[n++] = j;
+        counts[u] = n;
+    }
+}
+
+/* ---------------------------------------------------------------------------
+ * a6 [INF]: masked causal attention, written as the explicit definition (no
+ * tiling, no online rescaling).  For query token r in block i of head h:
+ *   s_c = scale * q_r . k_c   for every key c <= r whose block is active in
+ *                             mask[b,h,i,:]
+ *   O_r = sum_c softmax(s)_c v_c,  LSE_r = log(sum_c exp(s_c)).
+ * Rows with no admissible key get O_r = 0 and LSE_r = -inf.
+ * units: n_units triples (b, h, i); o: f64 [n_units, 64, d];
+ * lse: f64 [n_units, 64].  q: bf16 [B,Hq,S,d]; k, v: bf16 [B,Hkv,S,d].
+ * ------------------------------------------------------------------------- */
+void oracle_masked_attention(const uint16_t *q, const uint16_t *k,
+                             const uint16_t *v, int B, int Hq, int Hkv, int S,
+                             int d, const uint8_t *mask, double scale,
+                             const int32_t *units, int n_units, double *o,
+                             double *lse)
+{
+    const int nb = S / SEER_ORACLE_BLOCK;
+    const int g = Hq / Hkv;
+    (void)B;
+#pragma omp parallel
+    {
+        double *s = (double *)malloc(sizeof(double) * (size_t)S);
+        double *qrow = (double *)malloc(sizeof(double) * (size_t)d);
+#pragma omp for schedule(dynamic, 1)
+        for (int u = 0; u < n_units; ++u) {
+            const int b = units[3 * u], h = units[3 * u + 1], i = units[3 * u + 2];
+            const uint8_t *mrow = mask + (((long long)b * Hq + h) * nb + i) * nb;
+            const uint16_t *qh = q + ((long long)b * Hq + h) * S * d;
+            const uint16_t *kh = k + ((long long)b * Hkv + h / g) * S * d;
+            const uint16_t *vh = v + ((long long)b * Hkv + h / g) * S * d;
+            for (int t = 0; t < SEER_ORACLE_BLOCK; ++t) {
+                const int r = i * SEER_ORACLE_BLOCK + t;
+                double *orow = o + ((long long)u * SEER_ORACLE_BLOCK + t) * d;
+                for (int c = 0; c < d; ++c)
+                    qrow[c] = bf16_to_f64(qh[(long long)r * d + c]);
+                double m = -INFINITY;
+                for (int c = 0; c <= r; ++c) {
+                    if (!mrow[c / SEER_ORACLE_BLOCK])
+                        continue;
+                    double dot = 0.0;
+                    for (int e = 0; e < d; ++e)
+                        dot += qrow[e] * bf16_to_f64(kh[(long long)c * d + e]);
+                    s[c] = dot * scale;
+                    if (s[c] > m)
+                        m = s[c];
+                }
+                for (int e = 0; e < d; ++e)
+                    orow[e] = 0.0;
+                if (m == -INFINITY) {
+                    lse[(long long)u * SEER_ORACLE_BLOCK + t] = -INFINITY;
+                    continue;
+                }
+                double l = 0.0;
+                for (int c = 0; c <= r; ++c) {
+                    if (!mrow[c / SEER_ORACLE_BLOCK])
+                        continue;
+                    const double p = exp(s[c] - m);
+                    l += p;
+                    for (int e = 0; e < d; ++e)
+                        orow[e] += p * bf16_to_f64(vh[(long long)c * d + e]);
+                }
+                for (int e = 0; e < d; ++e)
+                    orow[e] /= l;
+                lse[(long long)u * SEER_ORACLE_BLOCK + t] = m + log(l);
+            }
+        }
+        free(s);
+        free(qrow);
+    }
+}
+
+/* ---------------------------------------------------------------------------
+ * a7 [FIG8]: dense causal attention output O together with the 2D max-pooled
+ * attention map.  Written from the definition the figure computes: with
+ * P_rc = softmax_{c<=r}(scale * q_r . k_c),
+ *   A[i, j] = max_{r in block i, c in block j, c <= r} P_rc,   0 for j > i.
+ * (The figure's two passes give exactly this: exp(rowmax_j - m_r)/l_r is the
+ * largest P_rc of row r inside block j, and colmax takes the max over r.)
+ * units: n_units triples (b, h, i); o: f64 [n_units, 64, d];
+ * A: f64 [n_units, nb].
+ * ------------------------------------------------------------------------- */
+void oracle_pooled_map(const uint16_t *q, const uint16_t *k, const uint16_t *v,
+                       int B, int Hq, int Hkv, int S, int d, double scale,
+                       const int32_t *units, int n_units, double *o, double *A)
+{
+    const int nb = S / SEER_ORACLE_BLOCK;
+    const int g = Hq / Hkv;
+    (void)B;
+#pragma omp parallel
+    {
+        double *s = (double *)malloc(sizeof(double) * (size_t)S);
+        double *qrow = (double *)malloc(sizeof(double) * (size_t)d);
+#pragma omp for schedule(dynamic, 1)
+        for (int u = 0; u < n_units; ++u) {
+            const int b = units[3 * u], h = units[3 * u + 1], i = units[3 * u + 2];
+            const uint16_t *qh = q + ((long long)b * Hq + h) * S * d;
+            const uint16_t *kh = k + ((long long)b * Hkv + h / g) * S * d;
+            const uint16_t *vh = v + ((long long)b * Hkv + h / g) * S * d;
+            double *arow = A + (long long)u * nb;
+            for (int j = 0; j < nb; ++j)
+                arow[j] = 0.0;
+            for (int t = 0; t < SEER_ORACLE_BLOCK; ++t) {
+                const int r = i * SEER_ORACLE_BLOCK + t;
+                double *orow = o + ((long long)u * SEER_ORACLE_BLOCK + t) * d;
+                for (int c = 0; c < d; ++c)
+                    qrow[c] = bf16_to_f64(qh[(long long)r * d + c]);
+                double m = -INFINITY;
+                for (int c = 0; c <= r; ++c) {
+                    double dot = 0.0;
+                    for (int e = 0; e < d; ++e)
+                        dot += qrow[e] * bf16_to_f64(kh[(long long)c * d + e]);
+                    s[c] = dot * scale;
+                    if (s[c] > m)
+                        m = s[c];
+                }
+                double l = 0.0;
+                for (int c = 0; c <= r; ++c)
+                    l += exp(s[c] - m);
+                for (int e = 0; e < d; ++e)
+                    orow[e] = 0.0;
+                for (int c = 0; c <= r; ++c) {
+                    const double p = exp(s[c] - m) / l;
+                    const int j = c / SEER_ORACLE_BLOCK;
+                    if (p > arow[j])
+                        arow[j] = p;
+                    for (int e = 0; e < d; ++e)
+                        orow[e] += p * bf16_to_f64(vh[(long long)c * d + e]);
+                }
+            }
+        }
+        free(s);
+        free(qrow);
+    }
+}

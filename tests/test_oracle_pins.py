@@ -1,0 +1,380 @@
+"""Pins for the fp64 oracle: closed forms, invariants and brute force.
+
+Each check compares the oracle with something other than itself: a value the
+mathematics fixes (closed forms, invariants) or an independent brute-force
+formulation (full matrices in numpy, complex-number rotation, sorting).  The
+sizes are tiny so the whole file runs in seconds on the CPU.
+"""
+import math
+
+import numpy as np
+import pytest
+
+from conftest import bits_to_f64, f64_to_bits
+
+BLOCK = 64
+
+
+def rng(seed):
+    return np.random.default_rng(seed)
+
+
+def rand_bits(shape, seed, scale=1.0, shift=0.0):
+    return f64_to_bits(rng(seed).standard_normal(shape) * scale + shift)
+
+
+# --------------------------------------------------------------------------- a1
+def test_pool_constant_blocks(oracle):
+    B, H, S, d = 1, 2, 256, 8
+    vals = np.arange(B * H * (S // BLOCK), dtype=np.float64).reshape(B, H, S // BLOCK) * 0.25
+    x = np.repeat(vals[..., None], BLOCK, axis=-1).reshape(B, H, S)[..., None].repeat(d, -1)
+    out = oracle.pool_avg(f64_to_bits(x))
+    np.testing.assert_array_equal(out, np.repeat(vals[..., None], d, -1))
+
+
+def test_pool_brute_force(oracle):
+    bits = rand_bits((2, 3, 192, 16), 1)
+    x = bits_to_f64(bits)
+    want = x.reshape(2, 3, 3, BLOCK, 16).sum(axis=3) / BLOCK
+    np.testing.assert_allclose(oracle.pool_avg(bits), want, rtol=0, atol=1e-14)
+
+
+# ------------------------------------------------------------------------- RoPE
+def test_rope_identity_at_block_zero(oracle):
+    x = rng(2).standard_normal(16)
+    np.testing.assert_array_equal(oracle.block_rope(x, 0, 5e5), x)
+
+
+def test_rope_closed_form_basis_vectors(oracle):
+    dg, theta = 8, 100.0
+    for t in range(dg // 2):
+        for p in (1, 3, 17):
+            e = np.zeros(dg)
+            e[t] = 1.0
+            y = oracle.block_rope(e, p, theta)
+            ang = p * theta ** (-2.0 * t / dg)
+            want = np.zeros(dg)
+            want[t] = math.cos(ang)
+            want[t + dg // 2] = math.sin(ang)
+            np.testing.assert_allclose(y, want, atol=1e-15)
+
+
+def test_rope_matches_complex_rotation(oracle):
+    dg, theta = 32, 5e5
+    x = rng(3).standard_normal(dg)
+    for p in (0, 1, 5, 511, 2047):
+        z = x[: dg // 2] + 1j * x[dg // 2:]
+        freqs = theta ** (-2.0 * np.arange(dg // 2) / dg)
+        z = z * np.exp(1j * p * freqs)
+        want = np.concatenate([z.real, z.imag])
+        np.testing.assert_allclose(oracle.block_rope(x, p, theta), want, atol=1e-12)
+
+
+def test_rope_norm_and_relative_position(oracle):
+    dg, theta = 64, 5e5
+    a, b = rng(4).standard_normal((2, dg))
+    for p in (1, 100, 1000):
+        assert abs(np.linalg.norm(oracle.block_rope(a, p, theta)) - np.linalg.norm(a)) < 1e-12
+    dot = lambda i, j: oracle.block_rope(a, i, theta) @ oracle.block_rope(b, j, theta)
+    for i, j, s in ((5, 2, 7), (40, 40, 3), (9, 0, 100)):
+        assert abs(dot(i, j) - dot(i + s, j + s)) < 1e-10
+
+
+# ------------------------------------------------------------------------ a2/a3
+def test_project_identity_weight(oracle):
+    B, H, nb, d = 1, 2, 3, 8
+    xp = rng(5).standard_normal((B, H, nb, d))
+    w = f64_to_bits(np.eye(d))
+    out = oracle.project_rope(xp, w, 5e5)          # shared weight (stride 0)
+    for i in range(nb):
+        for h in range(H):
+            np.testing.assert_allclose(out[0, h, i], oracle.block_rope(xp[0, h, i], i, 5e5), atol=1e-14)
+    np.testing.assert_array_equal(out[:, :, 0], xp[:, :, 0])
+
+
+def test_project_per_head_weights_brute_force(oracle):
+    B, H, nb, d, dg = 2, 3, 4, 16, 8
+    xp = rng(6).standard_normal((B, H, nb, d))
+    wbits = rand_bits((H, d, dg), 7, scale=0.2)
+    w = bits_to_f64(wbits)
+    out = oracle.project_rope(xp, wbits, 1e4)
+    for b in range(B):
+        for h in range(H):
+            for i in range(nb):
+                y = xp[b, h, i] @ w[h]
+                z = (y[: dg // 2] + 1j * y[dg // 2:]) * np.exp(1j * i * 1e4 ** (-2.0 * np.arange(dg // 2) / dg))
+                np.testing.assert_allclose(out[b, h, i], np.concatenate([z.real, z.imag]), atol=1e-12)
+
+
+def test_block_softmax_rows_and_zero_query(oracle):
+    B, Hq, Hkv, nb, dg = 1, 4, 2, 9, 8
+    kt = rng(8).standard_normal((B, Hkv, nb, dg))
+    s = oracle.block_softmax(np.zeros((B, Hq, nb, dg)), kt)
+    for i in range(nb):
+        np.testing.assert_allclose(s[..., i, : i + 1], 1.0 / (i + 1), atol=1e-15)
+        assert np.all(s[..., i, i + 1:] == 0)
+    qt = rng(9).standard_normal((B, Hq, nb, dg)) * 3
+    s = oracle.block_softmax(qt, kt)
+    np.testing.assert_allclose(s.sum(-1), 1.0, atol=1e-13)
+    assert np.all(np.triu(s[0, 0], 1) == 0)
+
+
+def test_block_softmax_brute_force_gqa(oracle):
+    B, Hq, Hkv, nb, dg = 2, 6, 2, 7, 16
+    qt = rng(10).standard_normal((B, Hq, nb, dg))
+    kt = rng(11).standard_normal((B, Hkv, nb, dg))
+    got = oracle.block_softmax(qt, kt)
+    kfull = np.repeat(kt, Hq // Hkv, axis=1)
+    logits = np.einsum("bhid,bhjd->bhij", qt, kfull) / math.sqrt(dg)
+    logits = np.where(np.tril(np.ones((nb, nb), bool)), logits, -np.inf)
+    e = np.exp(logits - logits.max(-1, keepdims=True))
+    np.testing.assert_allclose(got, e / e.sum(-1, keepdims=True), rtol=1e-12, atol=1e-15)
+
+
+def _np_gate(q, k, wq, wk, theta):
+    """Independent numpy formulation of the gate (reshape-mean, matmul, complex rotation)."""
+    B, Hq, S, d = q.shape
+    Hkv, nb = k.shape[1], S // BLOCK
+    dg = wq.shape[-1]
+    qp = q.reshape(B, Hq, nb, BLOCK, d).mean(3)
+    kp = k.reshape(B, Hkv, nb, BLOCK, d).mean(3)
+    qt = np.einsum("bhid,hde->bhie", qp, wq)
+    kt = np.einsum("bhid,hde->bhie", kp, wk)
+    rot = np.exp(1j * np.arange(nb)[:, None] * theta ** (-2.0 * np.arange(dg // 2) / dg)[None, :])
+
+    def apply(x):
+        z = (x[..., : dg // 2] + 1j * x[..., dg // 2:]) * rot
+        return np.concatenate([z.real, z.imag], -1)
+
+    qt, kt = apply(qt), apply(kt)
+    kt = np.repeat(kt, Hq // Hkv, axis=1)
+    lg = np.einsum("bhie,bhje->bhij", qt, kt) / math.sqrt(dg)
+    lg = np.where(np.tril(np.ones((nb, nb), bool)), lg, -np.inf)
+    e = np.exp(lg - lg.max(-1, keepdims=True))
+    return e / e.sum(-1, keepdims=True)
+
+
+def test_gate_scores_brute_force(oracle):
+    B, Hq, Hkv, S, d, dg = 1, 4, 2, 512, 32, 16
+    qb, kb = rand_bits((B, Hq, S, d), 12, scale=4.0), rand_bits((B, Hkv, S, d), 13, scale=4.0, shift=0.5)
+    wqb, wkb = rand_bits((Hq, d, dg), 14, scale=0.5), rand_bits((Hkv, d, dg), 15, scale=0.5)
+    got = oracle.gate_scores(qb, kb, wqb, wkb, theta=1e2)
+    want = _np_gate(bits_to_f64(qb), bits_to_f64(kb), bits_to_f64(wqb), bits_to_f64(wkb), 1e2)
+    np.testing.assert_allclose(got, want, rtol=1e-11, atol=1e-15)
+
+
+def test_gate_scores_zero_key_weight_is_uniform(oracle):
+    B, Hq, Hkv, S, d, dg = 1, 2, 1, 384, 16, 8
+    qb, kb = rand_bits((B, Hq, S, d), 16), rand_bits((B, Hkv, S, d), 17)
+    wqb = rand_bits((Hq, d, dg), 18)
+    wkb = f64_to_bits(np.zeros((Hkv, d, dg)))
+    s = oracle.gate_scores(qb, kb, wqb, wkb)
+    nb = S // BLOCK
+    for i in range(nb):
+        np.testing.assert_allclose(s[..., i, : i + 1], 1.0 / (i + 1), atol=1e-15)
+
+
+# --------------------------------------------------------------------------- a4
+def test_threshold_strict_forced_and_monotone(oracle):
+    nb = 12
+    s = np.abs(rng(19).standard_normal((1, 2, nb, nb))).astype(np.float32)
+    s = np.tril(s)
+    tau = float(s[0, 0, 7, 3])                          # an exact score value
+    m = oracle.block_mask(s, "threshold", tau, force_first=False, force_diag=False)
+    assert m[0, 0, 7, 3] == 0                           # strict >
+    np.testing.assert_array_equal(m, (s > np.float32(tau)) & np.tril(np.ones((nb, nb), bool)))
+    mf = oracle.block_mask(s, "threshold", 1e9)
+    want = np.zeros((nb, nb), np.uint8)
+    want[:, 0] = 1
+    want[np.arange(nb), np.arange(nb)] = 1
+    np.testing.assert_array_equal(mf[0, 1], want)
+    prev = None
+    for t in (0.0, 0.2, 0.5, 1.0, 2.0):
+        cur = oracle.block_mask(s, "threshold", t)
+        if prev is not None:
+            assert np.all(cur <= prev)
+        prev = cur
+    assert np.all(np.triu(prev[0, 0], 1) == 0)
+
+
+def _np_topk_mask(s, k_row, ff, fd):
+    B, H, nb, _ = s.shape
+    out = np.zeros_like(s, dtype=np.uint8)
+    for b in range(B):
+        for h in range(H):
+            for i in range(nb):
+                forced = set()
+                if ff:
+                    forced.add(0)
+                if fd:
+                    forced.add(i)
+                k = min(max(int(k_row[i]), len(forced)), i + 1)
+                rest = sorted((j for j in range(i + 1) if j not in forced),
+                              key=lambda j: (-float(s[b, h, i, j]), j))
+                for j in list(forced) + rest[: k - len(forced)]:
+                    out[b, h, i, j] = 1
+    return out
+
+
+@pytest.mark.parametrize("ff,fd", [(True, True), (False, False), (True, False), (False, True)])
+def test_topk_exact_count_and_brute_force(oracle, ff, fd):
+    nb = 16
+    s = np.tril(np.abs(rng(20).standard_normal((2, 3, nb, nb)))).astype(np.float32)
+    s[0, 0, 10, :6] = 0.5                                # ties: lower j must win
+    k_row = np.array([oracle.topk_count(0.3, i, 0) for i in range(nb)], np.int32)
+    m = oracle.block_mask(s, "topk", k_row=k_row, force_first=ff, force_diag=fd)
+    np.testing.assert_array_equal(m, _np_topk_mask(s, k_row, ff, fd))
+    for i in range(nb):
+        nf = len(({0} if ff else set()) | ({i} if fd else set()))
+        assert np.all(m[..., i, :].sum(-1) == min(max(k_row[i], nf), i + 1))
+
+
+def test_topk_count_closed_form(oracle):
+    assert oracle.topk_count(0.1, 0, 1) == 1
+    assert oracle.topk_count(0.1, 9, 2) == 2        # ceil(1.0) = 1 -> clamped to 2 forced
+    assert oracle.topk_count(0.1, 99, 2) == 10
+    assert oracle.topk_count(0.1, 100, 2) == 11     # ceil(10.1)
+    assert oracle.topk_count(1.0, 511, 2) == 512
+    assert oracle.topk_count(0.5, 7, 0) == 4
+    assert oracle.topk_count(2.0, 3, 0) == 4        # clamped to i + 1
+
+
+# --------------------------------------------------------------------------- a5
+def test_compact_lists(oracle):
+    nb = 10
+    m = (rng(21).random((2, 3, nb, nb)) < 0.4).astype(np.uint8) * np.tril(np.ones((nb, nb), np.uint8))
+    lists, counts = oracle.compact(m)
+    np.testing.assert_array_equal(counts, m.sum(-1))
+    for b in range(2):
+        for h in range(3):
+            for i in range(nb):
+                off = i * (i + 1) // 2
+                np.testing.assert_array_equal(lists[b, h, off: off + counts[b, h, i]], np.nonzero(m[b, h, i])[0])
+
+
+# --------------------------------------------------------------------------- a6
+def _np_masked_attention(q, k, v, mask, scale):
+    """Full-matrix formulation: token-level mask from the block mask, then softmax."""
+    B, Hq, S, d = q.shape
+    g = Hq // k.shape[1]
+    kf, vf = np.repeat(k, g, 1), np.repeat(v, g, 1)
+    tok = np.repeat(np.repeat(mask.astype(bool), BLOCK, -1), BLOCK, -2)
+    tok &= np.tril(np.ones((S, S), bool))
+    s = np.einsum("bhrd,bhcd->bhrc", q, kf) * scale
+    s = np.where(tok, s, -np.inf)
+    mx = s.max(-1, keepdims=True)
+    has = np.isfinite(mx)
+    p = np.where(has, np.exp(s - np.where(has, mx, 0)), 0.0)
+    l = p.sum(-1, keepdims=True)
+    o = np.where(has, np.einsum("bhrc,bhcd->bhrd", p, vf) / np.where(has, l, 1), 0.0)
+    lse = np.where(has[..., 0], (mx + np.log(np.where(has, l, 1)))[..., 0], -np.inf)
+    return o, lse
+
+
+def _as_units(o, B, H, nb, d):
+    return o.reshape(B * H * nb, BLOCK, d)
+
+
+def test_attention_random_mask_brute_force(oracle):
+    B, Hq, Hkv, S, d = 1, 4, 2, 384, 32
+    nb = S // BLOCK
+    qb, kb, vb = (rand_bits((B, h, S, d), 22 + i) for i, h in enumerate((Hq, Hkv, Hkv)))
+    m = (rng(25).random((B, Hq, nb, nb)) < 0.5).astype(np.uint8) * np.tril(np.ones((nb, nb), np.uint8))
+    m[0, 1, 3, :] = 0                      # a row with no active block at all
+    o, lse = oracle.masked_attention(qb, kb, vb, m)
+    wo, wl = _np_masked_attention(bits_to_f64(qb), bits_to_f64(kb), bits_to_f64(vb), m, 1 / math.sqrt(d))
+    np.testing.assert_allclose(o, _as_units(wo, B, Hq, nb, d), rtol=1e-10, atol=1e-12)
+    np.testing.assert_allclose(lse, wl.reshape(-1, BLOCK), rtol=1e-12)
+    assert np.all(o.reshape(B, Hq, nb, BLOCK, d)[0, 1, 3] == 0)
+
+
+def test_attention_density_one_is_dense_causal(oracle):
+    B, Hq, Hkv, S, d = 1, 2, 1, 256, 16
+    nb = S // BLOCK
+    qb, kb, vb = (rand_bits((B, h, S, d), 30 + i, scale=2.0) for i, h in enumerate((Hq, Hkv, Hkv)))
+    full = np.ones((B, Hq, nb, nb), np.uint8)
+    o, lse = oracle.masked_attention(qb, kb, vb, full, scale=0.3)
+    q, k, v = bits_to_f64(qb), bits_to_f64(kb), bits_to_f64(vb)
+    s = np.einsum("hrd,cd->hrc", q[0], k[0, 0]) * 0.3 + np.triu(np.full((S, S), -np.inf), 1)
+    p = np.exp(s - s.max(-1, keepdims=True))
+    want = (p / p.sum(-1, keepdims=True)) @ v[0, 0]
+    np.testing.assert_allclose(o.reshape(Hq, S, d), want, rtol=1e-10, atol=1e-12)
+
+
+def test_attention_all_diagonal_is_block_local(oracle):
+    B, Hq, Hkv, S, d = 1, 2, 2, 256, 16
+    nb = S // BLOCK
+    qb, kb, vb = (rand_bits((B, h, S, d), 40 + i) for i, h in enumerate((Hq, Hkv, Hkv)))
+    diag = np.broadcast_to(np.eye(nb, dtype=np.uint8), (B, Hq, nb, nb)).copy()
+    o, _ = oracle.masked_attention(qb, kb, vb, diag)
+    q, k, v = bits_to_f64(qb), bits_to_f64(kb), bits_to_f64(vb)
+    for h in range(Hq):
+        for i in range(nb):
+            sl = slice(i * BLOCK, (i + 1) * BLOCK)
+            s = q[0, h, sl] @ k[0, h, sl].T / 4.0 + np.triu(np.full((BLOCK, BLOCK), -np.inf), 1)
+            p = np.exp(s - s.max(-1, keepdims=True))
+            want = (p / p.sum(-1, keepdims=True)) @ v[0, h, sl]
+            np.testing.assert_allclose(o[h * nb + i], want, rtol=1e-10, atol=1e-12)
+
+
+def test_attention_zero_query_prefix_mean_and_constant_v(oracle):
+    B, Hq, Hkv, S, d = 1, 1, 1, 192, 8
+    nb = S // BLOCK
+    kb, vb = rand_bits((B, Hkv, S, d), 50), rand_bits((B, Hkv, S, d), 51)
+    qz = f64_to_bits(np.zeros((B, Hq, S, d)))
+    full = np.ones((B, Hq, nb, nb), np.uint8)
+    o, lse = oracle.masked_attention(qz, kb, vb, full)
+    v = bits_to_f64(vb)[0, 0]
+    want = np.cumsum(v, 0) / np.arange(1, S + 1)[:, None]
+    np.testing.assert_allclose(o.reshape(S, d), want, rtol=1e-12, atol=1e-14)
+    np.testing.assert_allclose(lse.reshape(S), np.log(np.arange(1, S + 1)), rtol=1e-14)
+    vc = f64_to_bits(np.full((B, Hkv, S, d), 1.5))
+    m = (rng(52).random((B, Hq, nb, nb)) < 0.5).astype(np.uint8) | np.eye(nb, dtype=np.uint8)
+    o, _ = oracle.masked_attention(rand_bits((B, Hq, S, d), 53), kb, vc, np.tril(m))
+    np.testing.assert_allclose(o, 1.5, rtol=1e-14)
+
+
+# --------------------------------------------------------------------------- a7
+def test_pooled_map_brute_force_and_bounds(oracle):
+    B, Hq, Hkv, S, d = 1, 2, 1, 320, 16
+    nb = S // BLOCK
+    qb, kb, vb = (rand_bits((B, h, S, d), 60 + i, scale=2.0) for i, h in enumerate((Hq, Hkv, Hkv)))
+    o, A = oracle.pooled_map(qb, kb, vb)
+    q, k, v = bits_to_f64(qb), bits_to_f64(kb), bits_to_f64(vb)
+    A = A.reshape(Hq, nb, nb)
+    for h in range(Hq):
+        s = q[0, h] @ k[0, 0].T / 4.0 + np.triu(np.full((S, S), -np.inf), 1)
+        p = np.exp(s - s.max(-1, keepdims=True))
+        p /= p.sum(-1, keepdims=True)
+        np.testing.assert_allclose(o.reshape(Hq, S, d)[h], p @ v[0, 0], rtol=1e-10, atol=1e-12)
+        pooled = p.reshape(nb, BLOCK, nb, BLOCK).max(axis=(1, 3))
+        np.testing.assert_allclose(A[h], pooled, rtol=1e-12, atol=0)
+    assert np.all(A[:, 0, 0] == 1.0)
+    assert np.all((A >= 0) & (A <= 1))
+    assert np.all(np.triu(A, 1) == 0)
+    for i in range(nb):
+        assert np.all(A[:, i].max(-1) >= 1.0 / (BLOCK * i + 1) - 1e-15)
+        assert np.all(A[:, i].sum(-1) >= 1.0 / BLOCK) and np.all(A[:, i].sum(-1) <= BLOCK)
+
+
+def test_pooled_map_zero_query_closed_form(oracle):
+    B, Hq, Hkv, S, d = 1, 1, 1, 256, 8
+    nb = S // BLOCK
+    qz = f64_to_bits(np.zeros((B, Hq, S, d)))
+    _, A = oracle.pooled_map(qz, rand_bits((B, Hkv, S, d), 70), rand_bits((B, Hkv, S, d), 71))
+    for i in range(nb):
+        np.testing.assert_allclose(A[i, : i + 1], 1.0 / (BLOCK * i + 1), rtol=1e-14)
+        assert np.all(A[i, i + 1:] == 0)
+
+
+def test_pooled_map_units_subset_matches_full(oracle):
+    B, Hq, Hkv, S, d = 2, 2, 1, 256, 8
+    nb = S // BLOCK
+    qb, kb, vb = (rand_bits((B, h, S, d), 80 + i) for i, h in enumerate((Hq, Hkv, Hkv)))
+    of, Af = oracle.pooled_map(qb, kb, vb)
+    units = np.array([[1, 1, 3], [0, 0, 0], [1, 0, 2]], np.int32)
+    o, A = oracle.pooled_map(qb, kb, vb, units=units)
+    for n, (b, h, i) in enumerate(units):
+        idx = (b * Hq + h) * nb + i
+        np.testing.assert_array_equal(o[n], of[idx])
+        np.testing.assert_array_equal(A[n], Af[idx])
