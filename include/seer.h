@@ -1,0 +1,201 @@
+/*
+ * seer.h — C ABI of libseer, a B200 (sm_100a) implementation of the
+ * SeerAttention long-context prefill hot path:
+ *
+ *   AttnGate soft scores  ->  threshold / per-row TopK block mask
+ *   ->  block-sparse causal FlashAttention prefill (GQA)
+ *   plus the companion pass that returns O and the 2D max-pooled map A.
+ *
+ * Sources (web pages about SeerAttention):
+ *  - "SeerAttention: Learning Intrinsic Sparse Attention in Your LLMs",
+ *    rebuttal: Weakness 2 (per-row TopK, [Seq/Block, TopK] indices, gate is
+ *    self-attention without V), Weakness 3 (pooling shapes), Weakness 4
+ *    (padding), Weakness 5 (inference kernel pseudocode), Q1 (block RoPE).
+ *  - "SeerAttention-Llama-3.1-8B-AttnGates" model card (threshold/TopK on
+ *    the soft scores drives a block-sparse FlashAttention kernel).
+ *  - "SeerAttention: Self-distilled Attention Gating for Efficient
+ *    Long-context Prefilling": Figure 8 (O plus max-pooled attention map),
+ *    Sec. 4 (block size 64).
+ *
+ * Conventions for every call:
+ *  - Tensors are caller-owned DEVICE memory, contiguous, row-major.  Q, K, V
+ *    and O are bf16 in [B, H, S, d] order (Hq heads for Q/O, Hkv for K/V;
+ *    query head h reads KV head h / (Hq/Hkv)).  Block size is fixed at 64.
+ *  - The library never allocates device memory.  Calls that need scratch
+ *    take a caller-provided workspace of at least seer_workspace_bytes().
+ *  - Every call is asynchronous on `stream` (a cudaStream_t; NULL = legacy
+ *    default stream).  Argument checks run on the host before any launch
+ *    and return an error without touching the device.  A launch failure
+ *    returns SEER_ERR_CUDA.  Errors found on the device (a bounded wait that
+ *    ran out) are recorded in a device status word and reported by
+ *    seer_check_status().
+ *  - seer_last_error() returns a thread-local text for the last failure.
+ *  - Supported: S % 64 == 0 (S >= 64), S/64 <= 16384, d in {64, 128},
+ *    Hq % Hkv == 0.  Other shapes return SEER_ERR_UNSUPPORTED.
+ */
+#ifndef SEER_H
+#define SEER_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define SEER_API __attribute__((visibility("default")))
+#else
+#define SEER_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum seer_status {
+    SEER_OK = 0,
+    SEER_ERR_INVALID_ARG = 1,  /* null/misaligned pointer, bad shape value  */
+    SEER_ERR_UNSUPPORTED = 2,  /* valid but not implemented (S%64, d, ...)  */
+    SEER_ERR_WORKSPACE = 3,    /* workspace missing or too small            */
+    SEER_ERR_CUDA = 4,         /* a CUDA runtime/driver call failed         */
+    SEER_ERR_TIMEOUT = 5,      /* a device-side bounded wait ran out        */
+    SEER_ERR_DEVICE = 6        /* another device-side check failed          */
+} seer_status;
+
+/* Problem shape.  nb = S / 64 query/key blocks. */
+typedef struct seer_shape {
+    int B, Hq, Hkv, S, d;
+} seer_shape;
+
+/* AttnGate parameters ("Learning Intrinsic Sparse Attention", rebuttal Q1 on
+ * AttnGate's RoPE and Weakness 3): per-head linear maps d -> d_gate (no bias),
+ * block RoPE at position = block index with base rope_theta, rotate-half
+ * pairs (t, t + d_gate/2).  Weights are bf16 [d, d_gate] row-major per head;
+ * *_head_stride is the element distance between consecutive heads' matrices
+ * (0 = one matrix shared by all heads).  d_gate must be even, 2..256. */
+typedef struct seer_gate_params {
+    int d_gate;
+    float rope_theta;
+    long long wq_head_stride;
+    long long wk_head_stride;
+} seer_gate_params;
+
+/* Mask modes ("SeerAttention-Llama-3.1-8B-AttnGates": threshold/TopK on the
+ * soft scores; "Learning Intrinsic Sparse Attention", Weakness 2: TopK is
+ * per row). */
+enum { SEER_MASK_THRESHOLD = 0, SEER_MASK_TOPK = 1 };
+
+typedef struct seer_mask_params {
+    int mode;                   /* SEER_MASK_THRESHOLD or SEER_MASK_TOPK            */
+    float threshold;            /* THRESHOLD: keep j <= i with score > threshold   */
+    double density;             /* TOPK: k_i = ceil(density * (i+1)), when neither  */
+                                /*       k_per_row nor k_fixed is given             */
+    int k_fixed;                /* TOPK: if > 0, k_i = k_fixed                      */
+    const int32_t *k_per_row;   /* TOPK: DEVICE int32 [nb] or NULL; overrides both  */
+    int force_first;            /* keep block 0 in every row (counts toward k_i)    */
+    int force_diag;             /* keep block i in row i (counts toward k_i)        */
+} seer_mask_params;
+
+/* which_call values for seer_workspace_bytes(). */
+enum {
+    SEER_CALL_GATE_SCORES = 0,
+    SEER_CALL_BLOCK_SPARSE_PREFILL = 1,
+    SEER_CALL_ATTN_POOLED_MAP = 2
+};
+
+/*
+ * seer_gate_scores — AttnGate soft scores.
+ * ("Learning Intrinsic Sparse Attention", rebuttal Weakness 3: pool along
+ * the sequence axis, [B, H, S/64, d], before the linear layer; Q1: block
+ * RoPE on the non-RoPE'd pooled Q/K; Weakness 2: softmax like attention
+ * without V; Question 2: rows sum to 1.)
+ *   Qp = mean over each 64-token block of q   (K likewise: average pooling)
+ *   Qt = RoPE_i(Qp @ Wq[h]),  Kt = RoPE_j(Kp @ Wk[h_kv])
+ *   scores[b,h,i,j] = softmax_{j<=i}(Qt_i . Kt_j / sqrt(d_gate)); 0 for j > i.
+ * q: bf16 [B,Hq,S,d]; k: bf16 [B,Hkv,S,d]; wq/wk: bf16 per the params;
+ * scores: fp32 [B,Hq,nb,nb] (fully written).  Workspace:
+ * seer_workspace_bytes(SEER_CALL_GATE_SCORES, shape) bytes, 256-B aligned.
+ */
+SEER_API seer_status seer_gate_scores(const seer_shape *shape, const void *q, const void *k,
+                             const void *wq, const void *wk, const seer_gate_params *gp,
+                             float *scores, void *workspace, size_t ws_bytes, void *stream);
+
+/*
+ * seer_block_mask — binary block mask from soft scores (threshold or per-row
+ * TopK).  TopK keeps exactly k_i = clamp(k_i, |forced|, i+1) blocks of row i:
+ * the forced blocks, then the largest scores, ties to the lower block index.
+ * scores: fp32 [B,Hq,nb,nb] (entries j > i are ignored; scores must not be
+ * NaN); mask: u8 [B,Hq,nb,nb], fully written, 0 for j > i.  No workspace.
+ * Given identical scores the mask is bit-exact across runs and with the
+ * reference definition.
+ */
+SEER_API seer_status seer_block_mask(const seer_shape *shape, const float *scores,
+                            const seer_mask_params *mp, uint8_t *mask, void *stream);
+
+/*
+ * seer_compact_mask — per (b, h, i) ascending list of active key blocks
+ * ("Learning Intrinsic Sparse Attention", Weakness 5: the kernel loops over
+ * the selected blocks by index; Weakness 2: [Seq/Block, TopK] indices).
+ * mask: u8 [B,Hq,nb,nb] (entries j > i ignored).  lists: int32
+ * [B,Hq,nb*(nb+1)/2], causal-packed: row i starts at i*(i+1)/2 and holds
+ * counts[b,h,i] entries (the rest of its i+1 slots are left untouched).
+ * counts: int32 [B,Hq,nb].  No workspace.
+ */
+SEER_API seer_status seer_compact_mask(const seer_shape *shape, const uint8_t *mask, int32_t *lists,
+                              int32_t *counts, void *stream);
+
+/*
+ * seer_block_sparse_prefill — block-sparse causal attention, GQA
+ * ("Learning Intrinsic Sparse Attention", Weakness 5 pseudocode: per query
+ * block, online softmax over the selected key blocks only).  For query token
+ * r in block i of head h:  O_r = sum_c softmax(scale * q_r.k_c) v_c over keys
+ * c <= r whose block is active in mask[b,h,i,:]; LSE_r = log sum exp.
+ * Rows with no admissible key get O_r = 0 and LSE_r = -inf.
+ * q: bf16 [B,Hq,S,d], k/v: bf16 [B,Hkv,S,d], mask: u8 [B,Hq,nb,nb]
+ * (entries j > i ignored), o: bf16 [B,Hq,S,d], lse: fp32 [B,Hq,S] or NULL.
+ * softmax_scale <= 0 selects 1/sqrt(d).  q, k, v, o must be 16-B aligned.
+ * Workspace: seer_workspace_bytes(SEER_CALL_BLOCK_SPARSE_PREFILL) (may be 0;
+ * workspace may then be NULL).
+ */
+SEER_API seer_status seer_block_sparse_prefill(const seer_shape *shape, const void *q, const void *k,
+                                      const void *v, const uint8_t *mask, float softmax_scale,
+                                      void *o, float *lse, void *workspace, size_t ws_bytes,
+                                      void *stream);
+
+/*
+ * seer_attn_pooled_map — dense causal attention returning O and the 2D
+ * max-pooled attention map ("SeerAttention: Self-distilled Attention Gating",
+ * Figure 8: store the block row max r_ij, then a_ij = exp(r_ij - m_i)/l_i and
+ * A_ij = colmax(a_ij)):
+ *   A[b,h,i,j] = max_{r in block i, c in block j, c <= r} P_rc, 0 for j > i,
+ * with P the causal softmax of scale * q.k.  A is not row-normalised.
+ * q/k/v/o as above; A: fp32 [B,Hq,nb,nb] (fully written).  Workspace:
+ * seer_workspace_bytes(SEER_CALL_ATTN_POOLED_MAP, shape) bytes (holds the
+ * per-row block maxima of the queries in flight).
+ */
+SEER_API seer_status seer_attn_pooled_map(const seer_shape *shape, const void *q, const void *k,
+                                 const void *v, float softmax_scale, void *o, float *A,
+                                 void *workspace, size_t ws_bytes, void *stream);
+
+/* Workspace bytes a call needs for `shape` (0 for SEER_CALL_BLOCK_SPARSE_PREFILL).
+ * Returns 0 and sets the last error for an invalid shape or call id. */
+SEER_API size_t seer_workspace_bytes(int which_call, const seer_shape *shape);
+
+/* Synchronise `stream`, read and clear the device status word.  Returns
+ * SEER_OK, SEER_ERR_TIMEOUT, SEER_ERR_DEVICE or SEER_ERR_CUDA. */
+SEER_API seer_status seer_check_status(void *stream);
+
+/* Upper bound, in nanoseconds, on any single device-side wait of the
+ * attention kernels (default 2e9).  A wait that runs out sets the device
+ * status to SEER_ERR_TIMEOUT and the kernel exits cleanly.  0 means give up
+ * at the first unsatisfied poll (used to test the timeout path). */
+SEER_API void seer_set_wait_timeout_ns(unsigned long long ns);
+
+/* Thread-local description of the last failure ("" if none). */
+SEER_API const char *seer_last_error(void);
+
+/* Library version string. */
+SEER_API const char *seer_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SEER_H */

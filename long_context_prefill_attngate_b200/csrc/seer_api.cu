@@ -1,0 +1,345 @@
+// seer_api.cu — the C ABI (include/seer.h): host-side argument checks,
+// workspace sizing, tensor-map creation and kernel launches.  No device
+// memory is ever allocated here; no host<->device copies are made except the
+// status-word read in seer_check_status().
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "../../include/seer.h"
+#include "seer_internal.h"
+#include "seer_ptx.cuh"
+
+namespace seer {
+
+// Device status word: kernels record timeouts / failed checks here through a
+// pointer (first error wins); seer_check_status() reads and clears it.
+__device__ int g_status_word;
+
+namespace {
+
+thread_local char g_err[512] = "";
+unsigned long long g_timeout_ns = 2000000000ull;
+
+seer_status fail(seer_status s, const char *fmt, ...)
+{
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_err, sizeof g_err, fmt, ap);
+    va_end(ap);
+    return s;
+}
+
+seer_status ok()
+{
+    g_err[0] = '\0';
+    return SEER_OK;
+}
+
+seer_status cuda_fail(cudaError_t e, const char *what)
+{
+    return fail(SEER_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+seer_status check_shape(const seer_shape *sh)
+{
+    if (sh == nullptr)
+        return fail(SEER_ERR_INVALID_ARG, "shape is NULL");
+    if (sh->B <= 0 || sh->Hq <= 0 || sh->Hkv <= 0 || sh->S <= 0 || sh->d <= 0)
+        return fail(SEER_ERR_INVALID_ARG, "shape fields must be positive (B=%d Hq=%d Hkv=%d S=%d d=%d)", sh->B,
+                    sh->Hq, sh->Hkv, sh->S, sh->d);
+    if (sh->Hq % sh->Hkv != 0)
+        return fail(SEER_ERR_INVALID_ARG, "Hq (%d) must be a multiple of Hkv (%d)", sh->Hq, sh->Hkv);
+    if (sh->S % kBlock != 0)
+        return fail(SEER_ERR_UNSUPPORTED, "S (%d) must be a multiple of 64", sh->S);
+    if (sh->d != 64 && sh->d != 128)
+        return fail(SEER_ERR_UNSUPPORTED, "head dim %d not supported (64 or 128)", sh->d);
+    if (sh->S / kBlock > kMaxNb)
+        return fail(SEER_ERR_UNSUPPORTED, "S/64 = %d exceeds %d", sh->S / kBlock, kMaxNb);
+    if ((long long)sh->B * sh->Hq > (1LL << 30) / kMaxNb)
+        return fail(SEER_ERR_UNSUPPORTED, "B*Hq too large");
+    return SEER_OK;
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int *status_ptr()
+{
+    // One address per device (the symbol lives in each device's copy of the module).
+    static std::mutex mu;
+    static int *cache[64] = {nullptr};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64)
+        return nullptr;
+    std::lock_guard<std::mutex> lk(mu);
+    if (cache[dev] == nullptr) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_status_word) != cudaSuccess)
+            return nullptr;
+        cache[dev] = static_cast<int *>(p);
+    }
+    return cache[dev];
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn()
+{
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+} // namespace
+
+// [B*H, S, d] bf16 viewed as a 3D tensor (d innermost); 64 x 64 boxes with
+// the 128-byte swizzle the MMA descriptors expect.
+bool make_tmap_bhsd(CUtensorMap *map, const void *base, int BH, int S, int d)
+{
+    EncodeTiledFn fn = encode_fn();
+    if (fn == nullptr)
+        return false;
+    const cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)S, (cuuint64_t)BH};
+    const cuuint64_t strides[2] = {(cuuint64_t)d * 2, (cuuint64_t)S * d * 2};
+    const cuuint32_t box[3] = {64, 64, 1};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    const CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box,
+                          estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+} // namespace seer
+
+using namespace seer;
+
+extern "C" {
+
+const char *seer_version(void) { return "seer-b200 0.1.0 (sm_100a)"; }
+
+const char *seer_last_error(void) { return g_err; }
+
+void seer_set_wait_timeout_ns(unsigned long long ns) { g_timeout_ns = ns; }
+
+size_t seer_workspace_bytes(int which_call, const seer_shape *shape)
+{
+    if (check_shape(shape) != SEER_OK)
+        return 0;
+    const int nb = shape->S / kBlock;
+    switch (which_call) {
+    case SEER_CALL_GATE_SCORES:
+        return gate_workspace_bytes(shape->B, shape->Hq, shape->Hkv, shape->S, shape->d, 256);
+    case SEER_CALL_BLOCK_SPARSE_PREFILL:
+        return 0;
+    case SEER_CALL_ATTN_POOLED_MAP:
+        return sizeof(float) * (size_t)kMaxAttnCtas * nb * 128;
+    default:
+        fail(SEER_ERR_INVALID_ARG, "unknown call id %d", which_call);
+        return 0;
+    }
+}
+
+seer_status seer_gate_scores(const seer_shape *shape, const void *q, const void *k, const void *wq, const void *wk,
+                             const seer_gate_params *gp, float *scores, void *workspace, size_t ws_bytes,
+                             void *stream)
+{
+    seer_status st = check_shape(shape);
+    if (st != SEER_OK)
+        return st;
+    if (gp == nullptr || q == nullptr || k == nullptr || wq == nullptr || wk == nullptr || scores == nullptr)
+        return fail(SEER_ERR_INVALID_ARG, "seer_gate_scores: NULL argument");
+    if (gp->d_gate < 2 || gp->d_gate > 256 || (gp->d_gate & 1))
+        return fail(SEER_ERR_UNSUPPORTED, "d_gate %d must be even and in [2, 256]", gp->d_gate);
+    if (!(gp->rope_theta > 0.f) || !std::isfinite(gp->rope_theta))
+        return fail(SEER_ERR_INVALID_ARG, "rope_theta must be positive and finite");
+    if (gp->wq_head_stride < 0 || gp->wk_head_stride < 0)
+        return fail(SEER_ERR_INVALID_ARG, "weight head strides must be >= 0");
+    if (!aligned16(q) || !aligned16(k))
+        return fail(SEER_ERR_INVALID_ARG, "q and k must be 16-byte aligned");
+    if ((gp->d_gate % 4) != 0)
+        return fail(SEER_ERR_UNSUPPORTED, "d_gate %d must be a multiple of 4", gp->d_gate);
+    const size_t need = gate_workspace_bytes(shape->B, shape->Hq, shape->Hkv, shape->S, shape->d, gp->d_gate);
+    if (workspace == nullptr || ws_bytes < need)
+        return fail(SEER_ERR_WORKSPACE, "seer_gate_scores needs %zu workspace bytes, got %zu", need, ws_bytes);
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+        return fail(SEER_ERR_WORKSPACE, "workspace must be 256-byte aligned");
+    const cudaError_t e = launch_gate(shape->B, shape->Hq, shape->Hkv, shape->S, shape->d, gp->d_gate,
+                                      gp->rope_theta, q, k, wq, gp->wq_head_stride, wk, gp->wk_head_stride, scores,
+                                      workspace, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess)
+        return cuda_fail(e, "seer_gate_scores launch");
+    return ok();
+}
+
+seer_status seer_block_mask(const seer_shape *shape, const float *scores, const seer_mask_params *mp, uint8_t *mask,
+                            void *stream)
+{
+    seer_status st = check_shape(shape);
+    if (st != SEER_OK)
+        return st;
+    if (mp == nullptr || scores == nullptr || mask == nullptr)
+        return fail(SEER_ERR_INVALID_ARG, "seer_block_mask: NULL argument");
+    if (mp->mode != SEER_MASK_THRESHOLD && mp->mode != SEER_MASK_TOPK)
+        return fail(SEER_ERR_INVALID_ARG, "unknown mask mode %d", mp->mode);
+    if (mp->mode == SEER_MASK_TOPK && mp->k_per_row == nullptr && mp->k_fixed <= 0 &&
+        !(std::isfinite(mp->density) && mp->density >= 0.0))
+        return fail(SEER_ERR_INVALID_ARG, "TopK density must be finite and >= 0");
+    if (mp->mode == SEER_MASK_THRESHOLD && std::isnan(mp->threshold))
+        return fail(SEER_ERR_INVALID_ARG, "threshold is NaN");
+    const cudaError_t e = launch_mask(shape->B, shape->Hq, shape->S / kBlock, scores, mp->mode, mp->threshold,
+                                      mp->density, mp->k_fixed, mp->k_per_row, mp->force_first ? 1 : 0,
+                                      mp->force_diag ? 1 : 0, mask, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess)
+        return cuda_fail(e, "seer_block_mask launch");
+    return ok();
+}
+
+seer_status seer_compact_mask(const seer_shape *shape, const uint8_t *mask, int32_t *lists, int32_t *counts,
+                              void *stream)
+{
+    seer_status st = check_shape(shape);
+    if (st != SEER_OK)
+        return st;
+    if (mask == nullptr || lists == nullptr || counts == nullptr)
+        return fail(SEER_ERR_INVALID_ARG, "seer_compact_mask: NULL argument");
+    const cudaError_t e =
+        launch_compact(shape->B, shape->Hq, shape->S / kBlock, mask, lists, counts, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess)
+        return cuda_fail(e, "seer_compact_mask launch");
+    return ok();
+}
+
+static seer_status attention_common(const char *name, const seer_shape *shape, const void *q, const void *k,
+                                    const void *v, void *o)
+{
+    seer_status st = check_shape(shape);
+    if (st != SEER_OK)
+        return st;
+    if (q == nullptr || k == nullptr || v == nullptr || o == nullptr)
+        return fail(SEER_ERR_INVALID_ARG, "%s: NULL q/k/v/o", name);
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o))
+        return fail(SEER_ERR_INVALID_ARG, "%s: q, k, v, o must be 16-byte aligned", name);
+    return SEER_OK;
+}
+
+seer_status seer_block_sparse_prefill(const seer_shape *shape, const void *q, const void *k, const void *v,
+                                      const uint8_t *mask, float softmax_scale, void *o, float *lse, void *workspace,
+                                      size_t ws_bytes, void *stream)
+{
+    (void)workspace;
+    (void)ws_bytes;
+    seer_status st = attention_common("seer_block_sparse_prefill", shape, q, k, v, o);
+    if (st != SEER_OK)
+        return st;
+    if (mask == nullptr)
+        return fail(SEER_ERR_INVALID_ARG, "seer_block_sparse_prefill: NULL mask");
+    if (std::isnan(softmax_scale) || std::isinf(softmax_scale))
+        return fail(SEER_ERR_INVALID_ARG, "softmax_scale must be finite");
+    int *status = status_ptr();
+    if (status == nullptr)
+        return fail(SEER_ERR_CUDA, "cannot resolve the device status word");
+    AttnLaunch a{};
+    a.B = shape->B;
+    a.Hq = shape->Hq;
+    a.Hkv = shape->Hkv;
+    a.S = shape->S;
+    a.d = shape->d;
+    a.nb = shape->S / kBlock;
+    const float scale = softmax_scale > 0.f ? softmax_scale : 1.0f / sqrtf((float)shape->d);
+    a.scale_log2 = scale * 1.4426950408889634f;
+    a.mask = mask;
+    a.o = o;
+    a.lse = lse;
+    a.q = q;
+    a.k = k;
+    a.v = v;
+    a.map_mode = false;
+    a.timeout_ns = g_timeout_ns;
+    a.status = status;
+    const cudaError_t e = launch_attention(a, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess)
+        return cuda_fail(e, "seer_block_sparse_prefill launch");
+    return ok();
+}
+
+seer_status seer_attn_pooled_map(const seer_shape *shape, const void *q, const void *k, const void *v,
+                                 float softmax_scale, void *o, float *A, void *workspace, size_t ws_bytes,
+                                 void *stream)
+{
+    seer_status st = attention_common("seer_attn_pooled_map", shape, q, k, v, o);
+    if (st != SEER_OK)
+        return st;
+    if (A == nullptr)
+        return fail(SEER_ERR_INVALID_ARG, "seer_attn_pooled_map: NULL A");
+    if (std::isnan(softmax_scale) || std::isinf(softmax_scale))
+        return fail(SEER_ERR_INVALID_ARG, "softmax_scale must be finite");
+    const int nb = shape->S / kBlock;
+    const int grid = attn_grid_size(shape->B, shape->Hq, shape->Hkv, nb);
+    const size_t need = sizeof(float) * (size_t)grid * nb * 128;
+    if (workspace == nullptr || ws_bytes < need)
+        return fail(SEER_ERR_WORKSPACE, "seer_attn_pooled_map needs %zu workspace bytes, got %zu", need, ws_bytes);
+    int *status = status_ptr();
+    if (status == nullptr)
+        return fail(SEER_ERR_CUDA, "cannot resolve the device status word");
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    cudaError_t e = cudaMemsetAsync(A, 0, sizeof(float) * (size_t)shape->B * shape->Hq * nb * nb, s);
+    if (e != cudaSuccess)
+        return cuda_fail(e, "seer_attn_pooled_map memset");
+    AttnLaunch a{};
+    a.B = shape->B;
+    a.Hq = shape->Hq;
+    a.Hkv = shape->Hkv;
+    a.S = shape->S;
+    a.d = shape->d;
+    a.nb = nb;
+    const float scale = softmax_scale > 0.f ? softmax_scale : 1.0f / sqrtf((float)shape->d);
+    a.scale_log2 = scale * 1.4426950408889634f;
+    a.o = o;
+    a.A = A;
+    a.rscratch = static_cast<float *>(workspace);
+    a.q = q;
+    a.k = k;
+    a.v = v;
+    a.map_mode = true;
+    a.timeout_ns = g_timeout_ns;
+    a.status = status;
+    e = launch_attention(a, s);
+    if (e != cudaSuccess)
+        return cuda_fail(e, "seer_attn_pooled_map launch");
+    return ok();
+}
+
+seer_status seer_check_status(void *stream)
+{
+    cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess)
+        return cuda_fail(e, "seer_check_status sync");
+    int v = 0;
+    e = cudaMemcpyFromSymbol(&v, g_status_word, sizeof(int));
+    if (e != cudaSuccess)
+        return cuda_fail(e, "seer_check_status read");
+    if (v != 0) {
+        const int zero = 0;
+        cudaMemcpyToSymbol(g_status_word, &zero, sizeof(int));
+        if (v == kStatusTimeout)
+            return fail(SEER_ERR_TIMEOUT, "a device-side wait ran out");
+        return fail(SEER_ERR_DEVICE, "device-side check failed (code %d)", v);
+    }
+    return ok();
+}
+
+} // extern "C"

@@ -1,0 +1,50 @@
+// seer_internal.h — declarations shared by the library's .cu files (host side).
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+namespace seer {
+
+constexpr int kBlock = 64;            // block size of gate, mask and kernels
+constexpr int kMaxNb = 16384;         // S <= 1M tokens
+constexpr int kMaxAttnCtas = 296;     // 2 resident CTAs on each of 148 SMs
+constexpr int kAttnThreads = 224;     // 4 softmax warps + TMA + MMA + list builder
+
+struct AttnLaunch {
+    int B, Hq, Hkv, S, d, nb;
+    float scale_log2;             // softmax scale * log2(e)
+    const uint8_t *mask;          // sparse mode: [B,Hq,nb,nb]
+    void *o;                      // bf16 [B,Hq,S,d]
+    float *lse;                   // fp32 [B,Hq,S] or null
+    float *A;                     // map mode: fp32 [B,Hq,nb,nb]
+    float *rscratch;              // map mode: [grid][nb][128]
+    const void *q, *k, *v;
+    bool map_mode;
+    uint64_t timeout_ns;
+    int *status;                  // device status word
+};
+
+// Attention kernels (seer_attn.cu).  Returns a cudaError_t.
+cudaError_t launch_attention(const AttnLaunch &p, cudaStream_t stream);
+int attn_grid_size(int B, int Hq, int Hkv, int nb);
+
+// Gate kernels (seer_gate.cu).
+cudaError_t launch_gate(int B, int Hq, int Hkv, int S, int d, int dg, float theta, const void *q,
+                        const void *k, const void *wq, long long wq_stride, const void *wk,
+                        long long wk_stride, float *scores, void *ws, cudaStream_t stream);
+size_t gate_workspace_bytes(int B, int Hq, int Hkv, int S, int d, int dg);
+
+// Mask / compaction kernels (seer_mask.cu).
+cudaError_t launch_mask(int B, int Hq, int nb, const float *scores, int mode, float threshold,
+                        double density, int k_fixed, const int32_t *k_per_row, int force_first,
+                        int force_diag, uint8_t *mask, cudaStream_t stream);
+cudaError_t launch_compact(int B, int Hq, int nb, const uint8_t *mask, int32_t *lists, int32_t *counts,
+                           cudaStream_t stream);
+
+// Tensor-map creation through the driver entry point (seer_api.cu).
+bool make_tmap_bhsd(CUtensorMap *map, const void *base, int BH, int S, int d);
+
+} // namespace seer

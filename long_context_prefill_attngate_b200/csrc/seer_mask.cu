@@ -1,0 +1,237 @@
+// seer_mask.cu — block mask from the gate's soft scores, and mask compaction.
+//
+// "SeerAttention-Llama-3.1-8B-AttnGates" model card: the binary block mask
+// comes from threshold/TopK on the gate's soft scores.  "SeerAttention:
+// Learning Intrinsic Sparse Attention in Your LLMs", rebuttal Weakness 2: TopK
+// is applied per row (not globally) and the kept indices form a
+// [Seq/Block, TopK] tensor; Weakness 5: the sparse kernel loads blocks by
+// index.
+//
+// The mask must be bit-exact given identical scores, so every decision is a
+// plain comparison of fp32 values (k_i for a density is ceil(density*(i+1))
+// in double, as on the host).  TopK uses an exact radix select on the
+// order-preserving integer image of each score, forced blocks ranking above
+// every score, ties broken toward the lower block index.
+#include <cuda_runtime.h>
+
+#include "seer_internal.h"
+
+namespace seer {
+
+namespace {
+
+constexpr int kThrThreads = 256;
+
+__global__ void __launch_bounds__(kThrThreads)
+    threshold_kernel(const float *__restrict__ scores, long long total, int nb, float thr, int ff, int fd,
+                     uint8_t *__restrict__ mask)
+{
+    for (long long e = (long long)blockIdx.x * kThrThreads + threadIdx.x; e < total;
+         e += (long long)gridDim.x * kThrThreads) {
+        const int j = (int)(e % nb);
+        const int i = (int)((e / nb) % nb);
+        uint8_t m = 0;
+        if (j <= i)
+            m = (scores[e] > thr) || (ff && j == 0) || (fd && j == i);
+        mask[e] = m;
+    }
+}
+
+// Order-preserving map float -> uint32 (larger float -> larger key); -0 == +0.
+__device__ __forceinline__ uint32_t float_key(float f)
+{
+    uint32_t u = __float_as_uint(f);
+    if ((u & 0x7FFFFFFFu) == 0)
+        u = 0;
+    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+constexpr int kTopThreads = 256;
+
+__device__ __forceinline__ int block_exclusive_scan(int v, int *sbuf, int *total)
+{
+    // 256 threads: warp scan + warp totals.
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    int incl = v;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const int t = __shfl_up_sync(0xffffffffu, incl, off);
+        if (lane >= off)
+            incl += t;
+    }
+    if (lane == 31)
+        sbuf[warp] = incl;
+    __syncthreads();
+    if (warp == 0) {
+        int w = lane < kTopThreads / 32 ? sbuf[lane] : 0;
+        int wi = w;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const int t = __shfl_up_sync(0xffffffffu, wi, off);
+            if (lane >= off)
+                wi += t;
+        }
+        if (lane < kTopThreads / 32)
+            sbuf[lane] = wi - w;
+        if (lane == kTopThreads / 32 - 1)
+            sbuf[kTopThreads / 32] = wi;
+    }
+    __syncthreads();
+    const int res = sbuf[warp] + incl - v;
+    *total = sbuf[kTopThreads / 32];
+    __syncthreads();
+    return res;
+}
+
+// One CTA per row (b, h, i).
+__global__ void __launch_bounds__(kTopThreads)
+    topk_kernel(const float *__restrict__ scores, int nb, double density, int k_fixed,
+                const int32_t *__restrict__ k_per_row, int ff, int fd, uint8_t *__restrict__ mask)
+{
+    extern __shared__ uint32_t keys[];        // nb entries
+    __shared__ int hist[256];
+    __shared__ int sbuf[kTopThreads / 32 + 1];
+    __shared__ uint32_t s_prefix;
+    __shared__ int s_remaining;
+    const long long row = blockIdx.x;
+    const int i = (int)(row % nb);
+    const float *srow = scores + row * nb;
+    uint8_t *mrow = mask + row * nb;
+    const int n = i + 1;
+    const int n_forced = (ff ? 1 : 0) + ((fd && !(ff && i == 0)) ? 1 : 0);
+    int k;
+    if (k_per_row != nullptr) {
+        k = k_per_row[i];
+    } else if (k_fixed > 0) {
+        k = k_fixed;
+    } else {
+        const double want = ceil(density * (double)(i + 1));
+        k = (want > (double)(i + 1)) ? (i + 1) : (int)want;
+    }
+    if (k < n_forced)
+        k = n_forced;
+    if (k > n)
+        k = n;
+    if (k == n) {
+        for (int j = threadIdx.x; j < nb; j += kTopThreads)
+            mrow[j] = j <= i ? 1 : 0;
+        return;
+    }
+    for (int j = threadIdx.x; j < n; j += kTopThreads) {
+        const bool forced = (ff && j == 0) || (fd && j == i);
+        keys[j] = forced ? 0xFFFFFFFFu : float_key(srow[j]);
+    }
+    if (threadIdx.x == 0) {
+        s_prefix = 0;
+        s_remaining = k;
+    }
+    __syncthreads();
+    // Radix select of the k-th largest key, 8 bits at a time from the top.
+    uint32_t prefix = 0, pmask = 0;
+    for (int shift = 24; shift >= 0; shift -= 8) {
+        for (int t = threadIdx.x; t < 256; t += kTopThreads)
+            hist[t] = 0;
+        __syncthreads();
+        for (int j = threadIdx.x; j < n; j += kTopThreads) {
+            const uint32_t kk = keys[j];
+            if ((kk & pmask) == prefix)
+                atomicAdd(&hist[(kk >> shift) & 255u], 1);
+        }
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            int rem = s_remaining;
+            int dgt = 255;
+            for (; dgt > 0; --dgt) {
+                if (hist[dgt] >= rem)
+                    break;
+                rem -= hist[dgt];
+            }
+            s_prefix = prefix | ((uint32_t)dgt << shift);
+            s_remaining = rem;
+        }
+        __syncthreads();
+        prefix = s_prefix;
+        pmask |= 255u << shift;
+    }
+    const uint32_t kth = prefix;               // the k-th largest key
+    const int need_eq = s_remaining;           // how many keys equal to kth to keep
+    // Keys > kth are kept; among keys == kth the lowest j's are kept.
+    const int chunk = (n + kTopThreads - 1) / kTopThreads;
+    const int jb = threadIdx.x * chunk;
+    const int je = min(n, jb + chunk);
+    int ties = 0;
+    for (int j = jb; j < je; ++j)
+        ties += keys[j] == kth;
+    int total;
+    int rank = block_exclusive_scan(ties, sbuf, &total);
+    for (int j = jb; j < je; ++j) {
+        const uint32_t kk = keys[j];
+        uint8_t m = kk > kth;
+        if (kk == kth) {
+            m = rank < need_eq;
+            ++rank;
+        }
+        mrow[j] = m;
+    }
+    for (int j = n + threadIdx.x; j < nb; j += kTopThreads)
+        mrow[j] = 0;
+}
+
+// One warp per row: ascending list of active blocks j <= i and its length.
+__global__ void __launch_bounds__(256)
+    compact_kernel(const uint8_t *__restrict__ mask, long long rows, int nb, long long tri, int32_t *__restrict__ lists,
+                   int32_t *__restrict__ counts)
+{
+    const long long row = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
+    if (row >= rows)
+        return;
+    const int lane = threadIdx.x & 31;
+    const int i = (int)(row % nb);
+    const long long bh = row / nb;
+    const uint8_t *mrow = mask + row * nb;
+    int32_t *out = lists + bh * tri + (long long)i * (i + 1) / 2;
+    int count = 0;
+    for (int j0 = 0; j0 <= i; j0 += 32) {
+        const int j = j0 + lane;
+        const bool a = j <= i && mrow[j] != 0;
+        const uint32_t bal = __ballot_sync(0xffffffffu, a);
+        if (a)
+            out[count + __popc(bal & ((1u << lane) - 1u))] = j;
+        count += __popc(bal);
+    }
+    if (lane == 0)
+        counts[row] = count;
+}
+
+} // namespace
+
+cudaError_t launch_mask(int B, int Hq, int nb, const float *scores, int mode, float threshold, double density,
+                        int k_fixed, const int32_t *k_per_row, int ff, int fd, uint8_t *mask, cudaStream_t stream)
+{
+    const long long rows = (long long)B * Hq * nb;
+    if (mode == 0) {
+        const long long total = rows * nb;
+        long long blocks = (total + kThrThreads - 1) / kThrThreads;
+        if (blocks > 148LL * 64)
+            blocks = 148LL * 64;
+        threshold_kernel<<<(unsigned)blocks, kThrThreads, 0, stream>>>(scores, total, nb, threshold, ff, fd, mask);
+        return cudaGetLastError();
+    }
+    const size_t smem = sizeof(uint32_t) * (size_t)nb;
+    cudaError_t e = cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess)
+        return e;
+    topk_kernel<<<(unsigned)rows, kTopThreads, smem, stream>>>(scores, nb, density, k_fixed, k_per_row, ff, fd, mask);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_compact(int B, int Hq, int nb, const uint8_t *mask, int32_t *lists, int32_t *counts,
+                           cudaStream_t stream)
+{
+    const long long rows = (long long)B * Hq * nb;
+    const long long tri = (long long)nb * (nb + 1) / 2;
+    compact_kernel<<<(unsigned)((rows + 7) / 8), 256, 0, stream>>>(mask, rows, nb, tri, lists, counts);
+    return cudaGetLastError();
+}
+
+} // namespace seer
