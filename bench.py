@@ -1,0 +1,450 @@
+"""Benchmark: SeerAttention prefill layer on B200.
+
+One step = the inference hot path of one attention layer on one batch of
+synthetic input: AttnGate scores -> per-row TopK mask -> block-sparse causal
+attention (GQA).  Default workload: Llama-3.1-8B-shaped layer (32 q-heads,
+8 kv-heads, head dim 128) at 32k tokens, TopK density 0.1 (first and diagonal
+blocks kept).  Reported value: active-block TFLOP/s of the whole step
+(4*64*64*d flops per active (head, query block, key block)), summed over ranks
+(weak scaling: every rank runs its own layer) over the max time across ranks.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+
+Prints ONE JSON line on rank 0.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "sparse prefill ms/layer & active-block TFLOP/s (% bf16 peak) vs density, 32k"
+UNIT = "TFLOP/s"
+BLOCK = 64
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def attn_flops(mask_sum: int, d: int) -> float:
+    return 4.0 * BLOCK * BLOCK * d * float(mask_sum)
+
+
+def profile_traffic(kernel_src: str, summary: str):
+    """DRAM bytes per launch from a committed ncu summary, if it was taken on
+    the current source of the kernel (sha256 recorded in the summary)."""
+    path = os.path.join(ROOT, "profiles", summary)
+    if not os.path.exists(path):
+        return None
+    sha = hashlib.sha256(open(os.path.join(ROOT, kernel_src), "rb").read()).hexdigest()[:16]
+    tb, src = None, None
+    for line in open(path):
+        if line.startswith("traffic_bytes_per_launch:"):
+            tb = float(line.split(":", 1)[1])
+        if line.startswith("kernel_source_sha256_16:"):
+            src = line.split(":", 1)[1].strip()
+    return tb if (tb is not None and src == sha) else None
+
+
+class ClockSampler:
+    """nvidia-smi clocks / throttle reasons sampled every 200 ms while running."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = os.path.join("/tmp", f"seer_clocks_{os.getpid()}.csv")
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        if self.proc is None or not os.path.exists(self.path):
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax = float(parts[2])
+            except ValueError:
+                continue
+            for nm, val in zip(names, parts[5:9]):
+                if val.lower().startswith("active"):
+                    reasons.add(nm)
+        os.unlink(self.path)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def dist_setup(n_gpus: int):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=600))
+    return world, rank, local
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world: int):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+# --------------------------------------------------------------------------- GPU arm
+def run_gpu(args, world, rank, local):
+    import numpy as np
+    import torch
+
+    import long_context_prefill_attngate_b200 as seer
+    from long_context_prefill_attngate_b200 import build as seer_build
+    from long_context_prefill_attngate_b200 import synthetic as syn
+
+    seer_build.build()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    w = syn.WORKLOADS[args.workload]
+    x = syn.make_inputs(w, seed=w.seed + 1000 * rank)
+    pk, pk_kind = peaks()
+    stream = torch.cuda.current_stream()
+
+    q, k, v = (x[n].to(dev) for n in ("q", "k", "v"))
+    wq, wk = x["wq"].to(dev), x["wk"].to(dev)
+    nb = w.nb
+    sh = seer.shape_of(q, k)
+    scores = torch.empty((w.B, w.Hq, nb, nb), dtype=torch.float32, device=dev)
+    mask = torch.empty((w.B, w.Hq, nb, nb), dtype=torch.uint8, device=dev)
+    o = torch.empty_like(q)
+    gws = torch.empty(seer.seer_workspace_bytes(seer.SEER_CALL_GATE_SCORES, sh), dtype=torch.uint8, device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)   # > 126 MB L2
+
+    def gate_mask(density):
+        seer.seer_gate_scores(q, k, wq, wk, rope_theta=w.rope_theta, scores=scores, workspace=gws)
+        seer.seer_block_mask(scores, "topk", density=density, mask=mask, Hkv=w.Hkv, d=w.d)
+
+    def attention():
+        seer.seer_block_sparse_prefill(q, k, v, mask, o=o)
+
+    def timed_steps(density, steps, warmup):
+        ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(steps)]
+        for _ in range(warmup):
+            gate_mask(density)
+            attention()
+        torch.cuda.synchronize()
+        barrier(world)
+        torch.cuda.synchronize()
+        for s in range(steps):
+            flush.zero_()
+            e = ev[s]
+            e[0].record(stream)
+            seer.seer_gate_scores(q, k, wq, wk, rope_theta=w.rope_theta, scores=scores, workspace=gws)
+            e[1].record(stream)
+            seer.seer_block_mask(scores, "topk", density=density, mask=mask, Hkv=w.Hkv, d=w.d)
+            e[2].record(stream)
+            attention()
+            e[3].record(stream)
+        torch.cuda.synchronize()
+        barrier(world)
+        seer.seer_check_status()
+        gate = [e[0].elapsed_time(e[1]) for e in ev]
+        msk = [e[1].elapsed_time(e[2]) for e in ev]
+        att = [e[2].elapsed_time(e[3]) for e in ev]
+        step = [e[0].elapsed_time(e[3]) for e in ev]
+        return dict(gate=gate, mask=msk, attn=att, step=step)
+
+    # ---------------- headline: density from args (default 0.1), timed K steps
+    with ClockSampler(local) as clk:
+        t_wall0 = time.time()
+        res = timed_steps(args.density, args.steps, args.warmup)
+        t_wall = time.time() - t_wall0
+    clocks = clk.summary()
+    mask_sum = int(mask.sum(dtype=torch.int64).item())
+    flops = attn_flops(mask_sum, w.d)
+    density_meas = mask_sum / (w.B * w.Hq * nb * (nb + 1) / 2)
+    ms_step = statistics.mean(res["step"])
+    ms_attn = statistics.mean(res["attn"])
+    ms_gate = statistics.mean(res["gate"])
+    ms_mask = statistics.mean(res["mask"])
+    ms_step_max = max_over_ranks(ms_step, world)
+    value = world * flops / (ms_step_max * 1e-3) / 1e12
+    attn_tflops = flops / (ms_attn * 1e-3) / 1e12
+
+    # ---------------- density sweep (attention only; 1.0 is the dense causal point)
+    sweep = []
+    if not args.no_sweep:
+        for dens in w.densities or (1.0, 0.5, 0.3, 0.2, 0.1):
+            r = timed_steps(dens, max(3, args.steps // 2), 2)
+            ms = statistics.median(r["attn"])
+            msum = int(mask.sum(dtype=torch.int64).item())
+            fl = attn_flops(msum, w.d)
+            ent = {"density_target": dens,
+                   "density": round(msum / (w.B * w.Hq * nb * (nb + 1) / 2), 4),
+                   "attn_ms": round(ms, 4), "step_ms": round(statistics.median(r["step"]), 4),
+                   "active_tflops": round(fl / (ms * 1e-3) / 1e12, 1),
+                   "frac_of_bf16_peak": round(fl / (ms * 1e-3) / 1e12 / pk["bf16_tflops"], 4)}
+            if dens == 1.0:
+                fa = 4.0 * w.S * w.S * w.d * w.Hq * w.B / 2
+                ent["fa_convention_tflops"] = round(fa / (ms * 1e-3) / 1e12, 1)
+            sweep.append(ent)
+        # restore the headline mask for the e2e leg
+        gate_mask(args.density)
+
+    # ---------------- pooled-map companion pass (Figure 8) on the same layer
+    pooled = None
+    if not args.no_map:
+        A = torch.empty((w.B, w.Hq, nb, nb), dtype=torch.float32, device=dev)
+        mws = torch.empty(seer.seer_workspace_bytes(seer.SEER_CALL_ATTN_POOLED_MAP, sh), dtype=torch.uint8,
+                          device=dev)
+        om = torch.empty_like(q)
+        for _ in range(2):
+            seer.seer_attn_pooled_map(q, k, v, o=om, A=A, workspace=mws)
+        ts = []
+        for _ in range(3):
+            flush.zero_()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            seer.seer_attn_pooled_map(q, k, v, o=om, A=A, workspace=mws)
+            e1.record(stream)
+            torch.cuda.synchronize()
+            ts.append(e0.elapsed_time(e1))
+        seer.seer_check_status()
+        fl = attn_flops(w.B * w.Hq * nb * (nb + 1) // 2, w.d)
+        ms = statistics.median(ts)
+        pooled = {"ms": round(ms, 3), "active_tflops": round(fl / (ms * 1e-3) / 1e12, 1),
+                  "frac_of_bf16_peak": round(fl / (ms * 1e-3) / 1e12 / pk["bf16_tflops"], 4)}
+        del A, mws, om
+
+    # ---------------- e2e: pinned host inputs -> C ABI -> host output, per step
+    hq, hk, hv = (x[n].pin_memory() for n in ("q", "k", "v"))
+    hwq, hwk = x["wq"].pin_memory(), x["wk"].pin_memory()
+    ho = torch.empty(o.shape, dtype=o.dtype).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hwq, hwk))
+    d2h = ho.numel() * ho.element_size()
+    e2e_steps = max(3, args.steps // 2)
+
+    def e2e_step():
+        q.copy_(hq, non_blocking=True)
+        k.copy_(hk, non_blocking=True)
+        v.copy_(hv, non_blocking=True)
+        wq.copy_(hwq, non_blocking=True)
+        wk.copy_(hwk, non_blocking=True)
+        gate_mask(args.density)
+        attention()
+        ho.copy_(o, non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize()
+    barrier(world)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    seer.seer_check_status()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps, world)
+    e2e_value = world * flops / (e2e_ms * 1e-3) / 1e12
+
+    # ---------------- CPU baseline: the oracle on a bounded sample (rank 0, N=1)
+    cpu_baseline = None
+    if rank == 0 and world == 1 and not args.no_cpu:
+        cpu_baseline = oracle_sample(w, x, mask.cpu().numpy(), budget_s=args.cpu_budget)
+
+    traffic = profile_traffic("long_context_prefill_attngate_b200/csrc/seer_attn.cu",
+                              "attn_sparse_llama8b_32k_d0.1.md")
+    launches_per_step = 5 + 1 + 1   # gate: 2 pool + 2 project/RoPE + 1 softmax; mask: 1; attention: 1
+    out = {
+        "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms_step_max, 4), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "S": w.S, "d": w.d,
+                   "mask": "gate-topk", "density_target": args.density, "density": round(density_meas, 4),
+                   "d_gate": w.d_gate, "rope_theta": w.rope_theta,
+                   "l2": "flushed between timed steps (256 MiB write, outside the step events)",
+                   "parallelism": "replicas" if world > 1 else "single"},
+        "ms_layer_attention": round(ms_attn, 4), "ms_gate": round(ms_gate, 4), "ms_mask": round(ms_mask, 4),
+        "attention_active_tflops": round(attn_tflops, 1),
+        "roofline": {"bound": "tensor", "achieved": round(attn_tflops, 1), "peak": pk["bf16_tflops"],
+                     "unit": "TFLOP/s", "frac": round(attn_tflops / pk["bf16_tflops"], 4), "traffic": traffic,
+                     "peak_kind": f"{pk_kind} bf16 burst (cuBLAS)",
+                     "frac_of_sustained": round(attn_tflops / pk["bf16_tflops_sustained"], 4),
+                     "kernel": "attn_kernel<128,false> (seer_block_sparse_prefill)",
+                     "algorithmic_flops_per_launch": flops},
+        "density_sweep": sweep, "pooled_map": pooled,
+        "e2e": {"value": round(e2e_value, 2), "unit": UNIT, "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 3)},
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clocks, "cpu_baseline": cpu_baseline, "wall_s_timed_region": round(t_wall, 3),
+    }
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+
+
+def oracle_sample(w, x, mask_np, budget_s: float):
+    """Time the fp64 oracle on a bounded sample of query blocks of the workload."""
+    import numpy as np
+
+    import oracle
+    from long_context_prefill_attngate_b200 import synthetic as syn
+
+    oracle.build()
+    qb, kb, vb = (syn.bf16_bits(x[n]) for n in ("q", "k", "v"))
+    rng = np.random.default_rng(0)
+    nb = w.nb
+    units, flops, spent = [], 0.0, 0.0
+    t0 = time.time()
+    # grow the sample until the budget is used (units of 8 query blocks across heads)
+    while spent < budget_s:
+        batch = np.stack([np.zeros(8, np.int32), rng.integers(0, w.Hq, 8).astype(np.int32),
+                          rng.integers(0, nb, 8).astype(np.int32)], 1)
+        t = time.time()
+        oracle.masked_attention(qb, kb, vb, mask_np, units=batch)
+        spent += time.time() - t
+        units.append(batch)
+        flops += sum(attn_flops(int(mask_np[b, h, i].sum()), w.d) for b, h, i in batch)
+        if time.time() - t0 > 3 * budget_s:
+            break
+    cores = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
+    n = sum(len(u) for u in units)
+    return {"value": flops / spent / 1e12, "unit": UNIT, "cores": cores, "kind": "oracle",
+            "sample": f"{n} random (head, query block) units of {w.name} at the benchmark mask "
+                      f"(fp64 masked attention, {spent:.1f} s; gate/mask not included)"}
+
+
+# --------------------------------------------------------------------------- reference arm
+def run_reference(args, world, rank):
+    if rank != 0:
+        return
+    import numpy as np
+
+    import oracle
+    from long_context_prefill_attngate_b200 import synthetic as syn
+
+    oracle.build()
+    w = syn.WORKLOADS[args.workload]
+    x = syn.make_inputs(w)
+    qb, kb, vb = (syn.bf16_bits(x[n]) for n in ("q", "k", "v"))
+    # Mask from the oracle's own gate (fp64, cast to fp32 for the selection).
+    scores = oracle.gate_scores(qb, kb, syn.bf16_bits(x["wq"]), syn.bf16_bits(x["wk"]), theta=w.rope_theta)
+    mask = oracle.block_mask(scores.astype(np.float32), "topk", k_row=oracle.topk_counts(args.density, w.nb))
+    del scores
+    rng = np.random.default_rng(1)
+    per_step = max(1, args.ref_units)
+
+    def step():
+        units = np.stack([np.zeros(per_step, np.int32), rng.integers(0, w.Hq, per_step).astype(np.int32),
+                          rng.integers(0, w.nb, per_step).astype(np.int32)], 1)
+        t = time.time()
+        oracle.masked_attention(qb, kb, vb, mask, units=units)
+        dt = time.time() - t
+        return dt, sum(attn_flops(int(mask[b, h, i].sum()), w.d) for b, h, i in units)
+
+    for _ in range(args.warmup):
+        step()
+    tt, ff = 0.0, 0.0
+    for _ in range(args.steps):
+        dt, fl = step()
+        tt += dt
+        ff += fl
+    value = ff / tt / 1e12
+    cores = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
+    sample = (f"each step: {per_step} random (head, query block) units of {w.name}, fp64 masked attention "
+              f"with the oracle's own gate/TopK mask (computed once, untimed)")
+    out = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+           "steps": args.steps, "warmup": args.warmup, "ms_per_step": tt / args.steps * 1e3,
+           "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+           "data": "synthetic",
+           "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "S": w.S, "d": w.d,
+                      "mask": "gate-topk", "density_target": args.density},
+           "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample},
+           "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(out), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["native", "reference"], default="native")
+    ap.add_argument("--workload", default="llama8b_32k")
+    ap.add_argument("--density", type=float, default=0.1)
+    ap.add_argument("--no-sweep", action="store_true")
+    ap.add_argument("--no-map", action="store_true")
+    ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--cpu-budget", type=float, default=15.0)
+    ap.add_argument("--ref-units", type=int, default=16)
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "native":
+        args.warmup = 3
+    world, rank, local = dist_setup(args.gpus)
+    try:
+        if args.impl == "reference":
+            run_reference(args, world, rank)
+        else:
+            run_gpu(args, world, rank, local)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

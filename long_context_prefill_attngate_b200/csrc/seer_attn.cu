@@ -42,6 +42,7 @@ namespace seer {
 namespace {
 
 constexpr int kNStage = 2;            // K/V pipeline depth
+constexpr int kPrefetch = 4;          // L2 prefetch distance (key blocks)
 constexpr int kRows = 128;            // rows of one tile (two halves of 64)
 constexpr uint64_t kDrainNs = 200000000ull;
 
@@ -65,20 +66,26 @@ struct KParams {
     float *rscratch;
     uint64_t timeout_ns;
     int *status;
+    int nslots;              // independent tiles in flight per CTA (1 or 2)
+    int slot_bytes;          // shared memory per slot
 };
 
-// Tile order: level = 0 is the last query block (the longest causal rows).
-// Within a level: (b, kv head, lane); lane < g/2 pairs heads (2l, 2l+1) of
-// the group at the same query block; the last lane of an odd group pairs the
-// leftover head's blocks (i, i-1) on even levels and is empty on odd levels.
+// Tile order: KV-head major, so the CTAs running at any moment read the K/V
+// of one or two KV heads (a few tens of MB: L2-resident).  Inside a KV head,
+// level = 0 is the last query block (the longest causal rows) and levels go
+// down, so heavy tiles come first.  Within a level, lane < g/2 pairs heads
+// (2l, 2l+1) of the group at the same query block; the last lane of an odd
+// group pairs the leftover head's blocks (i, i-1) on even levels and is empty
+// on odd levels.
 __device__ __forceinline__ Unit decode_unit(const KParams &p, long long u)
 {
-    const long long per_level = (long long)p.B * p.Hkv * p.lanes;
-    const int level = (int)(u / per_level);
-    const int rem = (int)(u % per_level);
+    const long long per_group = (long long)p.nb * p.lanes;
+    const int group = (int)(u / per_group);          // b * Hkv + kvh
+    const int rem = (int)(u % per_group);
+    const int level = rem / p.lanes;
     const int lane = rem % p.lanes;
-    const int kvh = (rem / p.lanes) % p.Hkv;
-    const int b = rem / (p.lanes * p.Hkv);
+    const int kvh = group % p.Hkv;
+    const int b = group / p.Hkv;
     const int i = p.nb - 1 - level;
     Unit r;
     r.b = b;
@@ -122,13 +129,10 @@ struct Smem {
     static constexpr int kOffRed = kOffInfo + 2 * (int)sizeof(UnitInfo) + 16;
     static constexpr int kOffList = (kOffRed + 4 * 32 * 4 + 15) / 16 * 16;
     static constexpr int kBaseBytes = kOffList;
-    // K/V/Q tiles need 1024-B alignment for the 128-B swizzle pattern.
-    static int total_bytes(int nb)
-    {
-        int b = kBaseBytes + 2 * ((nb * 2 + 15) / 16 * 16) + 1024;
-        const int min_bytes = 80 * 1024;   // at most 2 CTAs per SM (TMEM: 2 x 256 columns)
-        return b < min_bytes ? min_bytes : b;
-    }
+    // One slot: Q, K/V ring, barriers, unit info and two list buffers; slots
+    // start on 1024-B boundaries (the 128-B swizzle pattern repeats every 1 KB).
+    static int slot_bytes(int nb) { return (kBaseBytes + 2 * ((nb * 2 + 15) / 16 * 16) + 1023) / 1024 * 1024; }
+    static int total_bytes(int nb, int nslots) { return nslots * slot_bytes(nb) + 1024; }
 };
 
 __device__ __forceinline__ float warp_max_transpose32(float (&v)[32], int lane)
@@ -157,7 +161,7 @@ __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, const W
 }
 
 template <int D, bool MAP>
-__global__ void __maxnreg__(144)
+__global__ void __launch_bounds__(kAttnThreads, 1)
     attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                 const __grid_constant__ CUtensorMap tmV, const KParams p)
 {
@@ -165,7 +169,16 @@ __global__ void __maxnreg__(144)
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     // Align the dynamic window to 1024 B.
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    const uint32_t sbase = smem_u32(smem);
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    // Two slots per CTA (one CTA per SM: TMEM allocation pins occupancy to 1).
+    // Each slot is an independent tile pipeline: warps 8s+0..3 softmax (TMEM
+    // lane quarters 0..3), 8s+4 TMA producer, 8s+5 MMA issuer, 8s+6 list
+    // builder, 8s+7 spare.  Slot s owns TMEM columns [256 s, 256 s + 256).
+    const int slot = warp >> 3;
+    const int wl = warp & 7;
+    uint8_t *ssm = smem + slot * p.slot_bytes;
+    const uint32_t sbase = smem_u32(ssm);
     const uint32_t sQ = sbase + L::kOffQ;
     const uint32_t sK = sbase + L::kOffK;
     const uint32_t sV = sbase + L::kOffV;
@@ -173,33 +186,34 @@ __global__ void __maxnreg__(144)
     auto bar = [&](int idx) -> uint32_t { return sBar + 8u * idx; };
     uint32_t *tmem_base_ptr = reinterpret_cast<uint32_t *>(smem + L::kOffMisc);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L::kOffMisc + 4);
-    UnitInfo *infos = reinterpret_cast<UnitInfo *>(smem + L::kOffInfo);
+    UnitInfo *infos = reinterpret_cast<UnitInfo *>(ssm + L::kOffInfo);
     const int list_stride = (p.nb * 2 + 15) / 16 * 8;   // uint16 entries per buffer
-    uint16_t *lists = reinterpret_cast<uint16_t *>(smem + L::kOffList);
-
-    const int warp = threadIdx.x >> 5;
-    const int lane = threadIdx.x & 31;
+    uint16_t *lists = reinterpret_cast<uint16_t *>(ssm + L::kOffList);
     const WaitCtx wc{abort_flag, p.timeout_ns, p.status};
 
     if (threadIdx.x == 0) {
-        mbar_init(bar(L::kBarQFull), 1);
-        mbar_init(bar(L::kBarQEmpty), 1);
-        for (int s = 0; s < kNStage; ++s) {
-            mbar_init(bar(L::kBarKFull + s), 1);
-            mbar_init(bar(L::kBarVFull + s), 1);
-            mbar_init(bar(L::kBarKEmpty + s), 1);
-            mbar_init(bar(L::kBarVEmpty + s), 1);
+        for (int sl = 0; sl < p.nslots; ++sl) {
+            const uint32_t sb0 = smem_u32(smem + sl * p.slot_bytes) + L::kOffBar;
+            auto bi = [&](int idx) -> uint32_t { return sb0 + 8u * idx; };
+            mbar_init(bi(L::kBarQFull), 1);
+            mbar_init(bi(L::kBarQEmpty), 1);
+            for (int s = 0; s < kNStage; ++s) {
+                mbar_init(bi(L::kBarKFull + s), 1);
+                mbar_init(bi(L::kBarVFull + s), 1);
+                mbar_init(bi(L::kBarKEmpty + s), 1);
+                mbar_init(bi(L::kBarVEmpty + s), 1);
+            }
+            for (int b = 0; b < 2; ++b) {
+                mbar_init(bi(L::kBarSFull + b), 1);
+                mbar_init(bi(L::kBarPFull + b), kRows);
+                mbar_init(bi(L::kBarListFull + b), 1);
+                mbar_init(bi(L::kBarListEmpty + b), 6);
+            }
+            mbar_init(bi(L::kBarODone + 0), 1);
+            mbar_init(bi(L::kBarODone + 1), 1);
+            mbar_init(bi(L::kBarOFree), kRows);
+            mbar_init(bi(L::kBarDrain), 1);
         }
-        for (int b = 0; b < 2; ++b) {
-            mbar_init(bar(L::kBarSFull + b), 1);
-            mbar_init(bar(L::kBarPFull + b), kRows);
-            mbar_init(bar(L::kBarListFull + b), 1);
-            mbar_init(bar(L::kBarListEmpty + b), 6);
-        }
-        mbar_init(bar(L::kBarODone + 0), 1);
-        mbar_init(bar(L::kBarODone + 1), 1);
-        mbar_init(bar(L::kBarOFree), kRows);
-        mbar_init(bar(L::kBarDrain), 1);
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -209,22 +223,27 @@ __global__ void __maxnreg__(144)
         tma_prefetch_desc(&tmV);
     }
     if (warp == 5) {
-        tmem_alloc(smem_u32(tmem_base_ptr), 256);
+        tmem_alloc(smem_u32(tmem_base_ptr), 512);
         tmem_relinquish();
         tc_fence_before();
     }
     __syncthreads();
     tc_fence_after();
-    const uint32_t tmem = *tmem_base_ptr;
+    const uint32_t tmem = *tmem_base_ptr + 256u * (uint32_t)slot;
     auto tS = [&](int b) -> uint32_t { return tmem + 64u * (uint32_t)b; };
     const uint32_t tO = tmem + 128u;
 
-    const long long stride = gridDim.x;
+    // Virtual CTA: this slot's share of the round-robin tile order.
+    const long long vcta = (long long)blockIdx.x * p.nslots + slot;
+    const long long stride = (long long)gridDim.x * p.nslots;
+    const bool slot_on = slot < p.nslots;
 
-    if (warp == 6) {
+    if (!slot_on) {
+        // idle slot (the tiles' shared memory did not fit twice)
+    } else if (wl == 6) {
         // ------------------------------------------------------------ list builder
         int n = 0;
-        for (long long u = blockIdx.x; u < p.n_units; u += stride) {
+        for (long long u = vcta; u < p.n_units; u += stride) {
             const Unit un = decode_unit(p, u);
             if (!un.valid)
                 continue;
@@ -290,13 +309,13 @@ __global__ void __maxnreg__(144)
                 mbar_arrive(bar(L::kBarListFull + lb));
             ++n;
         }
-    } else if (warp == 4) {
+    } else if (wl == 4) {
         // ------------------------------------------------------------ TMA producer
         if (lane == 0) {
             int n = 0, q_it = 0;
             long long kv_it = 0;
             bool ok = true;
-            for (long long u = blockIdx.x; u < p.n_units && ok; u += stride) {
+            for (long long u = vcta; u < p.n_units && ok; u += stride) {
                 const Unit un = decode_unit(p, u);
                 if (!un.valid)
                     continue;
@@ -346,6 +365,15 @@ __global__ void __maxnreg__(144)
                         for (int pn = 0; pn < L::kPanels; ++pn)
                             tma_load_3d(sV + s * L::kKVBytes + pn * L::kKVPanelBytes, &tmV, bar(L::kBarVFull + s),
                                         pn * 64, j * 64, zkv);
+                        // Warm L2 with the block kPrefetch positions ahead.
+                        if (t + kPrefetch < inf.count) {
+                            const int jp = lst[t + kPrefetch] & 0x3FFF;
+#pragma unroll
+                            for (int pn = 0; pn < L::kPanels; ++pn) {
+                                tma_prefetch_3d(&tmK, pn * 64, jp * 64, zkv);
+                                tma_prefetch_3d(&tmV, pn * 64, jp * 64, zkv);
+                            }
+                        }
                         ++kv_it;
                     }
                     if (!ok)
@@ -368,7 +396,7 @@ __global__ void __maxnreg__(144)
                     mbar_drain(bar(L::kBarQFull), (q_it - 1) & 1, kDrainNs);
             }
         }
-    } else if (warp == 5) {
+    } else if (wl == 5) {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
             constexpr uint32_t idS = idesc_bf16(128, 64, 0);
@@ -377,7 +405,7 @@ __global__ void __maxnreg__(144)
             long long kv_base = 0, sb = 0;
             bool ok = true;
             bool issued = false;
-            for (long long u = blockIdx.x; u < p.n_units && ok; u += stride) {
+            for (long long u = vcta; u < p.n_units && ok; u += stride) {
                 const Unit un = decode_unit(p, u);
                 if (!un.valid)
                     continue;
@@ -460,12 +488,12 @@ __global__ void __maxnreg__(144)
                 mbar_drain(bar(L::kBarDrain), 0, kDrainNs);
             }
         }
-    } else {
+    } else if (wl < 4) {
         // ------------------------------------------------------------ softmax / epilogue
-        const int row = threadIdx.x;          // 0..127 == TMEM lane
+        const int row = wl * 32 + lane;       // 0..127 == TMEM lane
         const int half = row >> 6;
         const int r_in = row & 63;
-        const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+        const uint32_t lane_off = (uint32_t)(wl * 32) << 16;
         int n = 0;
         long long sb = 0, pv_total = 0;
         // PV number n (counted over the CTA's lifetime) arrives on o_done[n & 1].
@@ -477,9 +505,9 @@ __global__ void __maxnreg__(144)
         auto wait_pv = [&](long long n_pv) -> bool {
             return warp_wait(bar(L::kBarODone + (int)(n_pv & 1)), (uint32_t)((n_pv >> 1) & 1), wc);
         };
-        float *rs = MAP ? p.rscratch + (size_t)blockIdx.x * p.nb * kRows : nullptr;
+        float *rs = MAP ? p.rscratch + (size_t)vcta * p.nb * kRows : nullptr;
         bool ok = true;
-        for (long long u = blockIdx.x; u < p.n_units && ok; u += stride) {
+        for (long long u = vcta; u < p.n_units && ok; u += stride) {
             const Unit un = decode_unit(p, u);
             if (!un.valid)
                 continue;
@@ -542,14 +570,14 @@ __global__ void __maxnreg__(144)
                         }
                         tc_fence_after();
 #pragma unroll 1
-                        for (int ch = 0; ch < D / 32; ++ch) {
-                            uint32_t ov[32];
-                            tmem_ld32(tO + lane_off + ch * 32, ov);
+                        for (int ch = 0; ch < D / 16; ++ch) {
+                            uint32_t ov[16];
+                            tmem_ld16(tO + lane_off + ch * 16, ov);
                             tmem_wait_ld();
 #pragma unroll
-                            for (int c = 0; c < 32; ++c)
+                            for (int c = 0; c < 16; ++c)
                                 ov[c] = __float_as_uint(__uint_as_float(ov[c]) * alpha);
-                            tmem_st32(tO + lane_off + ch * 32, ov);
+                            tmem_st16(tO + lane_off + ch * 16, ov);
                         }
                     }
                     m = m_new;
@@ -662,7 +690,7 @@ __global__ void __maxnreg__(144)
     __syncthreads();
     if (warp == 5) {
         tc_fence_after();
-        tmem_dealloc(tmem, 256);
+        tmem_dealloc(*tmem_base_ptr, 512);
     }
 }
 
@@ -690,13 +718,28 @@ cudaError_t launch_t(const AttnLaunch &a, cudaStream_t stream)
     p.rscratch = a.rscratch;
     p.timeout_ns = a.timeout_ns;
     p.status = a.status;
-    const int smem = Smem<D>::total_bytes(a.nb);
+    // Two tile slots per CTA when their shared memory fits (227 KB per CTA).
+    p.nslots = Smem<D>::total_bytes(a.nb, 2) <= 227 * 1024 ? 2 : 1;
+    p.slot_bytes = Smem<D>::slot_bytes(a.nb);
+    const int smem = Smem<D>::total_bytes(a.nb, p.nslots);
     auto kern = attn_kernel<D, MAP>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess)
         return e;
-    const int grid = attn_grid_size(a.B, a.Hq, a.Hkv, a.nb);
-    kern<<<grid, kAttnThreads, smem, stream>>>(tq, tk, tv, p);
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared);
+    if (e != cudaSuccess)
+        return e;
+    int dev = 0, sms = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess)
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    // One persistent CTA per SM (kernels that allocate TMEM run one CTA per SM).
+    const long long vctas = attn_grid_size(a.B, a.Hq, a.Hkv, a.nb);
+    long long grid = (vctas + p.nslots - 1) / p.nslots;
+    if (grid > sms)
+        grid = sms;
+    if (grid < 1)
+        grid = 1;
+    kern<<<(unsigned)grid, kAttnThreads, smem, stream>>>(tq, tk, tv, p);
     return cudaGetLastError();
 }
 

@@ -10,8 +10,8 @@ namespace seer {
 
 constexpr int kBlock = 64;            // block size of gate, mask and kernels
 constexpr int kMaxNb = 16384;         // S <= 1M tokens
-constexpr int kMaxAttnCtas = 296;     // 2 resident CTAs on each of 148 SMs
-constexpr int kAttnThreads = 224;     // 4 softmax warps + TMA + MMA + list builder
+constexpr int kMaxAttnCtas = 296;     // tile pipelines in flight: 2 slots x 148 SMs
+constexpr int kAttnThreads = 512;     // 2 slots x (4 softmax + TMA + MMA + list builder + spare) warps
 
 struct AttnLaunch {
     int B, Hq, Hkv, S, d, nb;
