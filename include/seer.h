@@ -174,6 +174,24 @@ SEER_API seer_status seer_attn_pooled_map(const seer_shape *shape, const void *q
                                  const void *v, float softmax_scale, void *o, float *A,
                                  void *workspace, size_t ws_bytes, void *stream);
 
+/*
+ * seer_gate_scores_noalloc — seer_gate_scores for callers that cannot
+ * allocate device memory (an embedding application whose pool owns all device
+ * memory, or a latency-critical path that must not call cudaMalloc).  The
+ * pages have no counterpart; it is a deployment convenience.  Same inputs,
+ * outputs and results as seer_gate_scores, but the workspace comes from a
+ * fixed 24 MiB device array inside the library (held by every GPU that loads
+ * the library until exit).  Shapes whose gate workspace
+ * (seer_workspace_bytes(SEER_CALL_GATE_SCORES) for the given d_gate) exceeds
+ * 24 MiB return SEER_ERR_UNSUPPORTED and launch nothing.  The first call on a
+ * device looks up the array's device address; make it before any stream
+ * capture.  All calls share the array: calls whose kernels overlap on the GPU
+ * race and must be ordered (one stream, or events).
+ */
+SEER_API seer_status seer_gate_scores_noalloc(const seer_shape *shape, const void *q, const void *k,
+                                              const void *wq, const void *wk, const seer_gate_params *gp,
+                                              float *scores, void *stream);
+
 /* Workspace bytes a call needs for `shape` (0 for SEER_CALL_BLOCK_SPARSE_PREFILL).
  * Returns 0 and sets the last error for an invalid shape or call id. */
 SEER_API size_t seer_workspace_bytes(int which_call, const seer_shape *shape);

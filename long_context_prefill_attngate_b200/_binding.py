@@ -37,7 +37,7 @@ BLOCK = 64
 EXPORTS = (
     "seer_gate_scores", "seer_block_mask", "seer_compact_mask", "seer_block_sparse_prefill",
     "seer_attn_pooled_map", "seer_workspace_bytes", "seer_check_status", "seer_set_wait_timeout_ns",
-    "seer_last_error", "seer_version",
+    "seer_last_error", "seer_version", "seer_gate_scores_noalloc",
 )
 
 
@@ -80,12 +80,13 @@ def lib() -> ctypes.CDLL:
             P, I, Z, F = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t, ctypes.c_float
             SP = ctypes.POINTER(seer_shape)
             L.seer_gate_scores.argtypes = [SP, P, P, P, P, ctypes.POINTER(seer_gate_params), P, P, Z, P]
+            L.seer_gate_scores_noalloc.argtypes = [SP, P, P, P, P, ctypes.POINTER(seer_gate_params), P, P]
             L.seer_block_mask.argtypes = [SP, P, ctypes.POINTER(seer_mask_params), P, P]
             L.seer_compact_mask.argtypes = [SP, P, P, P, P]
             L.seer_block_sparse_prefill.argtypes = [SP, P, P, P, P, F, P, P, P, Z, P]
             L.seer_attn_pooled_map.argtypes = [SP, P, P, P, F, P, P, P, Z, P]
-            for fn in ("seer_gate_scores", "seer_block_mask", "seer_compact_mask", "seer_block_sparse_prefill",
-                       "seer_attn_pooled_map", "seer_check_status"):
+            for fn in ("seer_gate_scores", "seer_gate_scores_noalloc", "seer_block_mask", "seer_compact_mask",
+                       "seer_block_sparse_prefill", "seer_attn_pooled_map", "seer_check_status"):
                 getattr(L, fn).restype = I
             L.seer_workspace_bytes.argtypes = [I, SP]
             L.seer_workspace_bytes.restype = Z
@@ -176,6 +177,29 @@ def seer_gate_scores(q, k, wq, wk, rope_theta: float = 5e5, scores=None, workspa
     gp = seer_gate_params(int(dg), float(rope_theta), int(wq_head_stride), int(wk_head_stride))
     _check(lib().seer_gate_scores(ctypes.byref(sh), _ptr(q), _ptr(k), _ptr(wq), _ptr(wk), ctypes.byref(gp),
                                   _ptr(scores), _ptr(workspace), wsb, _stream_ptr(stream)))
+    return scores
+
+
+def seer_gate_scores_noalloc(q, k, wq, wk, rope_theta: float = 5e5, scores=None, stream=None,
+                             wq_head_stride: int | None = None, wk_head_stride: int | None = None):
+    """seer_gate_scores without a workspace: the library's fixed scratch is used
+    (for callers that cannot allocate device memory; shapes needing more than
+    24 MiB of gate scratch raise SeerError)."""
+    torch = _torch()
+    _need(q.is_contiguous() and k.is_contiguous() and wq.is_contiguous() and wk.is_contiguous(),
+          "tensors must be contiguous")
+    sh = shape_of(q, k)
+    d, dg = sh.d, wq.shape[-1]
+    nb = sh.S // BLOCK
+    if wq_head_stride is None:
+        wq_head_stride = 0 if wq.dim() == 2 else d * dg
+    if wk_head_stride is None:
+        wk_head_stride = 0 if wk.dim() == 2 else d * dg
+    if scores is None:
+        scores = torch.empty((sh.B, sh.Hq, nb, nb), dtype=torch.float32, device=q.device)
+    gp = seer_gate_params(int(dg), float(rope_theta), int(wq_head_stride), int(wk_head_stride))
+    _check(lib().seer_gate_scores_noalloc(ctypes.byref(sh), _ptr(q), _ptr(k), _ptr(wq), _ptr(wk), ctypes.byref(gp),
+                                          _ptr(scores), _stream_ptr(stream)))
     return scores
 
 

@@ -106,6 +106,15 @@ EncodeTiledFn encode_fn()
 
 } // namespace
 
+seer_status set_last_error(seer_status s, const char *fmt, ...)
+{
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_err, sizeof g_err, fmt, ap);
+    va_end(ap);
+    return s;
+}
+
 // [B*H, S, d] bf16 viewed as a 3D tensor (d innermost); 64 x 64 boxes with
 // the 128-byte swizzle the MMA descriptors expect.
 bool make_tmap_bhsd(CUtensorMap *map, const void *base, int BH, int S, int d)

@@ -6,6 +6,8 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include "../../include/seer.h"
+
 namespace seer {
 
 constexpr int kBlock = 64;            // block size of gate, mask and kernels
@@ -43,6 +45,9 @@ cudaError_t launch_mask(int B, int Hq, int nb, const float *scores, int mode, fl
                         int force_diag, uint8_t *mask, cudaStream_t stream);
 cudaError_t launch_compact(int B, int Hq, int nb, const uint8_t *mask, int32_t *lists, int32_t *counts,
                            cudaStream_t stream);
+
+// Record the thread-local error text returned by seer_last_error() (seer_api.cu).
+seer_status set_last_error(seer_status s, const char *fmt, ...);
 
 // Tensor-map creation through the driver entry point (seer_api.cu).
 bool make_tmap_bhsd(CUtensorMap *map, const void *base, int BH, int S, int d);
