@@ -66,127 +66,226 @@ __global__ void __launch_bounds__(kPoolThreads) pool_kernel(const __nv_bfloat16 
     }
 }
 
-constexpr int kProjRows = 32;
-constexpr int kProjThreads = 256;
+constexpr int kProjRows = 64;
+constexpr int kProjThreads = 256;      // 16 x 16: rows ty + 16a, rotation pairs tx + 16b
+constexpr int kPStride = 4;            // padding (floats) of the shared rows
 
-// out[bh, i, :] = RoPE_i( xp[bh, i, :] @ W[h] ), rotate-half pairs (t, t+dg/2),
-// angle i * theta^(-2t/dg) evaluated in double precision.
+// out[bh, i, :] = RoPE_i( xp[bh, i, :] @ W[h] ) for 64 blocks i of one head.
+// Each thread owns 4 rows x 4 rotation pairs (t, t + dg/2), so both halves
+// of a pair are in its registers when the rotation is applied.  Angles
+// i * theta^(-2t/dg): frequencies in double once per CTA, angle formed and
+// reduced modulo 2*pi in double, the reduced angle through fp32 sincosf.
 __global__ void __launch_bounds__(kProjThreads)
     project_rope_kernel(const float *__restrict__ xp, int H, int nb, int d, const __nv_bfloat16 *__restrict__ w,
                         long long w_stride, int dg, double theta, float *__restrict__ out)
 {
-    extern __shared__ float psm[];
-    float *sx = psm;                                  // kProjRows x d
-    __nv_bfloat16 *sw = reinterpret_cast<__nv_bfloat16 *>(psm + kProjRows * d);   // d x dg
+    extern __shared__ float4 psm4[];
+    const int xs = d + kPStride;
+    float *sx = reinterpret_cast<float *>(psm4);           // kProjRows x xs
+    float *sw = sx + kProjRows * xs;                       // d x dg (fp32)
+    double *sfreq = reinterpret_cast<double *>(sw + d * dg);
     const int bh = blockIdx.y;
     const int h = bh % H;
     const int i0 = blockIdx.x * kProjRows;
     const int rows = min(kProjRows, nb - i0);
+    const int half = dg / 2;
     const __nv_bfloat16 *wh = w + (long long)h * w_stride;
     for (int e = threadIdx.x; e < d * dg; e += kProjThreads)
-        sw[e] = wh[e];
-    for (int e = threadIdx.x; e < rows * d; e += kProjThreads)
-        sx[e] = xp[((long long)bh * nb + i0) * d + e];
+        sw[e] = __bfloat162float(wh[e]);
+    const float *xb = xp + ((long long)bh * nb + i0) * d;
+    for (int e = threadIdx.x; e < kProjRows * d; e += kProjThreads) {
+        const int r = e / d, c = e % d;
+        sx[r * xs + c] = r < rows ? xb[e] : 0.f;
+    }
+    for (int t = threadIdx.x; t < half; t += kProjThreads)
+        sfreq[t] = pow(theta, -2.0 * (double)t / (double)dg);
     __syncthreads();
-    const int half = dg / 2;
-    for (int item = threadIdx.x; item < rows * half; item += kProjThreads) {
-        const int r = item / half;
-        const int t = item % half;
-        float y0 = 0.f, y1 = 0.f;
-        const float *xr = sx + r * d;
+    constexpr double kTwoPi = 6.283185307179586476925286766559;
+    const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
+    for (int t0 = 0; t0 < half; t0 += 64) {
+        float y0[4][4], y1[4][4];
+#pragma unroll
+        for (int a = 0; a < 4; ++a)
+#pragma unroll
+            for (int b = 0; b < 4; ++b)
+                y0[a][b] = y1[a][b] = 0.f;
+        int tcol[4];
+#pragma unroll
+        for (int b = 0; b < 4; ++b)
+            tcol[b] = min(t0 + tx + 16 * b, half - 1);
+#pragma unroll 2
         for (int c = 0; c < d; ++c) {
-            const float xv = xr[c];
-            y0 = fmaf(xv, __bfloat162float(sw[c * dg + t]), y0);
-            y1 = fmaf(xv, __bfloat162float(sw[c * dg + t + half]), y1);
+            float xv[4], w0[4], w1[4];
+#pragma unroll
+            for (int a = 0; a < 4; ++a)
+                xv[a] = sx[(ty + 16 * a) * xs + c];
+#pragma unroll
+            for (int b = 0; b < 4; ++b) {
+                w0[b] = sw[c * dg + tcol[b]];
+                w1[b] = sw[c * dg + tcol[b] + half];
+            }
+#pragma unroll
+            for (int a = 0; a < 4; ++a)
+#pragma unroll
+                for (int b = 0; b < 4; ++b) {
+                    y0[a][b] = fmaf(xv[a], w0[b], y0[a][b]);
+                    y1[a][b] = fmaf(xv[a], w1[b], y1[a][b]);
+                }
         }
-        const int i = i0 + r;
-        const double ang = (double)i * pow(theta, -2.0 * (double)t / (double)dg);
-        double sn, cs;
-        sincos(ang, &sn, &cs);
-        const float c = (float)cs, s = (float)sn;
-        float *o = out + ((long long)bh * nb + i) * dg;
-        o[t] = y0 * c - y1 * s;
-        o[t + half] = y1 * c + y0 * s;
+#pragma unroll
+        for (int a = 0; a < 4; ++a) {
+            const int r = ty + 16 * a;
+            if (r >= rows)
+                continue;
+            const int i = i0 + r;
+            float *o = out + ((long long)bh * nb + i) * dg;
+#pragma unroll
+            for (int b = 0; b < 4; ++b) {
+                const int t = t0 + tx + 16 * b;
+                if (t >= half)
+                    continue;
+                const double ang = (double)i * sfreq[t];
+                const double red = ang - rint(ang * (1.0 / kTwoPi)) * kTwoPi;
+                float sn, cs;
+                sincosf((float)red, &sn, &cs);
+                o[t] = y0[a][b] * cs - y1[a][b] * sn;
+                o[t + half] = y1[a][b] * cs + y0[a][b] * sn;
+            }
+        }
     }
 }
 
-constexpr int kSmRows = 16;          // query blocks per CTA
-constexpr int kSmCols = 64;          // key blocks per smem tile
-constexpr int kSmThreads = 256;
+constexpr int kLR = 64;              // query blocks per CTA
+constexpr int kLC = 64;              // key blocks per tile
+constexpr int kLThreads = 256;       // 16 x 16: rows ty + 16a, columns tx + 16b
+constexpr int kLPad = 4;             // row padding (floats): conflict-free float4 reads
 
-// Causal block logits + row softmax.  Each CTA owns kSmRows query blocks of
-// one head; raw logits are written to `scores`, then each row is turned into
-// its softmax in place (the row is still in L2), zeros for j > i.
-__global__ void __launch_bounds__(kSmThreads)
+// Causal block logits + row softmax for 64 query blocks of one head.  Each
+// thread computes 4 x 4 logits per 64 x 64 tile from float4 reads of the
+// shared Qt and Kt rows; raw logits (times 1/sqrt(dg)) go to `scores` while
+// each row's running max and exp-sum are kept online (the 16 threads sharing
+// a row reduce with shuffles).  A second pass over the same tiles writes
+// exp(x - m) / sum, and the entries j > i are set to 0.
+__global__ void __launch_bounds__(kLThreads)
     gate_softmax_kernel(const float *__restrict__ qt, const float *__restrict__ kt, int Hq, int Hkv, int nb, int dg,
                         float scale, float *__restrict__ scores)
 {
-    extern __shared__ float gsm[];
-    const int ks = dg + 4;                       // padded K row stride (conflict-free float4 reads)
-    float *sq = gsm;                             // kSmRows x dg
-    float *sk = gsm + kSmRows * dg;              // kSmCols x ks
-    const int bh = blockIdx.y;                   // b * Hq + h
+    extern __shared__ float4 gsm4[];
+    const int rs = dg + kLPad;
+    float *sq = reinterpret_cast<float *>(gsm4);           // kLR x rs
+    float *sk = sq + kLR * rs;                             // kLC x rs
+    const int bh = blockIdx.y;                             // b * Hq + h
     const int b = bh / Hq, h = bh % Hq;
     const int g = Hq / Hkv;
-    const int i0 = blockIdx.x * kSmRows;
-    const int rows = min(kSmRows, nb - i0);
+    const int i0 = blockIdx.x * kLR;
+    const int rows = min(kLR, nb - i0);
     const float *qbase = qt + ((long long)bh * nb + i0) * dg;
     const float *kbase = kt + ((long long)(b * Hkv + h / g) * nb) * dg;
-    for (int e = threadIdx.x; e < rows * dg; e += kSmThreads)
-        sq[e] = qbase[e];
+    const int dg4 = dg / 4;
+    for (int e = threadIdx.x; e < kLR * dg4; e += kLThreads) {
+        const int r = e / dg4, c4 = e % dg4;
+        const float4 v = r < rows ? reinterpret_cast<const float4 *>(qbase + (long long)r * dg)[c4]
+                                  : make_float4(0.f, 0.f, 0.f, 0.f);
+        *reinterpret_cast<float4 *>(sq + r * rs + 4 * c4) = v;
+    }
+    const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
     const int jlast = i0 + rows - 1;
-    const int jl = threadIdx.x % kSmCols;
-    const int rg = threadIdx.x / kSmCols;        // 0..3 -> rows rg, rg+4, rg+8, rg+12
-    for (int j0 = 0; j0 <= jlast; j0 += kSmCols) {
+    float m[4], ssum[4];
+#pragma unroll
+    for (int a = 0; a < 4; ++a) {
+        m[a] = -INFINITY;
+        ssum[a] = 0.f;
+    }
+    for (int j0 = 0; j0 <= jlast; j0 += kLC) {
         __syncthreads();
-        const int ncols = min(kSmCols, jlast + 1 - j0);
-        for (int e = threadIdx.x; e < ncols * dg; e += kSmThreads) {
-            const int jj = e / dg, cc = e % dg;
-            sk[jj * ks + cc] = kbase[(long long)(j0 + jj) * dg + cc];
+        const int ncols = min(kLC, jlast + 1 - j0);
+        for (int e = threadIdx.x; e < kLC * dg4; e += kLThreads) {
+            const int jj = e / dg4, c4 = e % dg4;
+            const float4 v = jj < ncols ? reinterpret_cast<const float4 *>(kbase + (long long)(j0 + jj) * dg)[c4]
+                                        : make_float4(0.f, 0.f, 0.f, 0.f);
+            *reinterpret_cast<float4 *>(sk + jj * rs + 4 * c4) = v;
         }
         __syncthreads();
-        const int j = j0 + jl;
-        if (jl < ncols) {
-            float acc[4] = {0.f, 0.f, 0.f, 0.f};
-            const float *kr = sk + jl * ks;
-            for (int c = 0; c < dg; c += 4) {
-                const float4 kv = *reinterpret_cast<const float4 *>(kr + c);
+        float acc[4][4];
 #pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    const float4 qv = *reinterpret_cast<const float4 *>(sq + (rg + 4 * q) * dg + c);
-                    acc[q] = fmaf(qv.x, kv.x, fmaf(qv.y, kv.y, fmaf(qv.z, kv.z, fmaf(qv.w, kv.w, acc[q]))));
+        for (int a = 0; a < 4; ++a)
+#pragma unroll
+            for (int c = 0; c < 4; ++c)
+                acc[a][c] = 0.f;
+#pragma unroll 2
+        for (int c = 0; c < dg; c += 4) {
+            float4 qv[4], kv[4];
+#pragma unroll
+            for (int a = 0; a < 4; ++a)
+                qv[a] = *reinterpret_cast<const float4 *>(sq + (ty + 16 * a) * rs + c);
+#pragma unroll
+            for (int bb = 0; bb < 4; ++bb)
+                kv[bb] = *reinterpret_cast<const float4 *>(sk + (tx + 16 * bb) * rs + c);
+#pragma unroll
+            for (int a = 0; a < 4; ++a)
+#pragma unroll
+                for (int bb = 0; bb < 4; ++bb)
+                    acc[a][bb] = fmaf(qv[a].x, kv[bb].x,
+                                      fmaf(qv[a].y, kv[bb].y, fmaf(qv[a].z, kv[bb].z, fmaf(qv[a].w, kv[bb].w, acc[a][bb]))));
+        }
+#pragma unroll
+        for (int a = 0; a < 4; ++a) {
+            const int r = ty + 16 * a;
+            const int i = i0 + r;
+            float tm = -INFINITY;
+#pragma unroll
+            for (int bb = 0; bb < 4; ++bb) {
+                const int j = j0 + tx + 16 * bb;
+                acc[a][bb] *= scale;
+                if (r < rows && j <= i) {
+                    scores[((long long)bh * nb + i) * nb + j] = acc[a][bb];
+                    tm = fmaxf(tm, acc[a][bb]);
                 }
             }
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                const int r = rg + 4 * q;
-                const int i = i0 + r;
+            for (int off = 1; off < 16; off <<= 1)
+                tm = fmaxf(tm, __shfl_xor_sync(0xffffffffu, tm, off));
+            const float mn = fmaxf(m[a], tm);
+            float ts = 0.f;
+#pragma unroll
+            for (int bb = 0; bb < 4; ++bb) {
+                const int j = j0 + tx + 16 * bb;
                 if (r < rows && j <= i)
-                    scores[((long long)bh * nb + i) * nb + j] = acc[q] * scale;
+                    ts += expf(acc[a][bb] - mn);
+            }
+#pragma unroll
+            for (int off = 1; off < 16; off <<= 1)
+                ts += __shfl_xor_sync(0xffffffffu, ts, off);
+            if (mn != -INFINITY) {
+                ssum[a] = (m[a] == -INFINITY ? 0.f : ssum[a] * expf(m[a] - mn)) + ts;
+                m[a] = mn;
             }
         }
     }
-    __syncthreads();
-    // Row softmax: one warp per row.
+    // Normalise: each thread rereads exactly the logits it wrote.
+    for (int j0 = 0; j0 <= jlast; j0 += kLC) {
+#pragma unroll
+        for (int a = 0; a < 4; ++a) {
+            const int r = ty + 16 * a;
+            const int i = i0 + r;
+            if (r >= rows)
+                continue;
+            const float inv = 1.0f / ssum[a];
+#pragma unroll
+            for (int bb = 0; bb < 4; ++bb) {
+                const int j = j0 + tx + 16 * bb;
+                if (j <= i) {
+                    float *p = scores + ((long long)bh * nb + i) * nb + j;
+                    *p = expf(*p - m[a]) * inv;
+                }
+            }
+        }
+    }
+    // Zeros above the diagonal.
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    for (int r = warp; r < rows; r += kSmThreads / 32) {
+    for (int r = warp; r < rows; r += kLThreads / 32) {
         const int i = i0 + r;
         float *row = scores + ((long long)bh * nb + i) * nb;
-        float mx = -INFINITY;
-        for (int j = lane; j <= i; j += 32)
-            mx = fmaxf(mx, row[j]);
-#pragma unroll
-        for (int off = 16; off; off >>= 1)
-            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
-        float sum = 0.f;
-        for (int j = lane; j <= i; j += 32)
-            sum += expf(row[j] - mx);
-#pragma unroll
-        for (int off = 16; off; off >>= 1)
-            sum += __shfl_xor_sync(0xffffffffu, sum, off);
-        const float inv = 1.0f / sum;
-        for (int j = lane; j <= i; j += 32)
-            row[j] = expf(row[j] - mx) * inv;
         for (int j = i + 1 + lane; j < nb; j += 32)
             row[j] = 0.f;
     }
@@ -229,7 +328,7 @@ cudaError_t launch_gate(int B, int Hq, int Hkv, int S, int d, int dg, float thet
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess)
         return e;
-    const size_t psmem = sizeof(float) * kProjRows * d + sizeof(__nv_bfloat16) * d * dg;
+    const size_t psmem = sizeof(float) * (kProjRows * (d + kPStride) + (size_t)d * dg) + sizeof(double) * (dg / 2) + 16;
     e = cudaFuncSetAttribute(project_rope_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)psmem);
     if (e != cudaSuccess)
         return e;
@@ -244,12 +343,12 @@ cudaError_t launch_gate(int B, int Hq, int Hkv, int S, int d, int dg, float thet
     e = cudaGetLastError();
     if (e != cudaSuccess)
         return e;
-    const size_t ssmem = sizeof(float) * (kSmRows * dg + kSmCols * (dg + 4));
+    const size_t ssmem = sizeof(float) * (size_t)(kLR + kLC) * (dg + kLPad);
     e = cudaFuncSetAttribute(gate_softmax_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ssmem);
     if (e != cudaSuccess)
         return e;
-    const dim3 sg((nb + kSmRows - 1) / kSmRows, B * Hq);
-    gate_softmax_kernel<<<sg, kSmThreads, ssmem, stream>>>(qt, kt, Hq, Hkv, nb, dg, 1.0f / sqrtf((float)dg), scores);
+    const dim3 sg((nb + kLR - 1) / kLR, B * Hq);
+    gate_softmax_kernel<<<sg, kLThreads, ssmem, stream>>>(qt, kt, Hq, Hkv, nb, dg, 1.0f / sqrtf((float)dg), scores);
     return cudaGetLastError();
 }
 

@@ -177,6 +177,94 @@ __global__ void __launch_bounds__(kTopThreads)
         mrow[j] = 0;
 }
 
+// k_i for row i (same rule as the host helper): k_per_row, else k_fixed, else
+// ceil(density * (i+1)) in double; clamped to [#forced, i+1].
+__device__ __forceinline__ int row_k(int i, double density, int k_fixed, const int32_t *k_per_row, int n_forced)
+{
+    int k;
+    if (k_per_row != nullptr) {
+        k = k_per_row[i];
+    } else if (k_fixed > 0) {
+        k = k_fixed;
+    } else {
+        const double want = ceil(density * (double)(i + 1));
+        k = (want > (double)(i + 1)) ? (i + 1) : (int)want;
+    }
+    if (k < n_forced)
+        k = n_forced;
+    if (k > i + 1)
+        k = i + 1;
+    return k;
+}
+
+// One warp per row (rows of up to 32 * PER candidates): lane L holds the keys
+// of blocks j = 32 e + L.  The k-th largest key is found bit by bit from the
+// top (32 counting rounds, one warp reduction each); keys above it are kept,
+// and among keys equal to it the lowest block indices, ranked with ballots.
+// Absent entries (j > i) hold key 0, below every real key.
+template <int PER>
+__global__ void __launch_bounds__(256)
+    topk_warp_kernel(const float *__restrict__ scores, long long rows, int nb, double density, int k_fixed,
+                     const int32_t *__restrict__ k_per_row, int ff, int fd, uint8_t *__restrict__ mask)
+{
+    const long long row = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
+    if (row >= rows)
+        return;
+    const int lane = threadIdx.x & 31;
+    const int i = (int)(row % nb);
+    const int n = i + 1;
+    const float *srow = scores + row * nb;
+    uint8_t *mrow = mask + row * nb;
+    const int n_forced = (ff ? 1 : 0) + ((fd && !(ff && i == 0)) ? 1 : 0);
+    const int k = row_k(i, density, k_fixed, k_per_row, n_forced);
+    if (k == n) {
+        for (int j = lane; j < nb; j += 32)
+            mrow[j] = j <= i ? 1 : 0;
+        return;
+    }
+    uint32_t key[PER];
+#pragma unroll
+    for (int e = 0; e < PER; ++e) {
+        const int j = 32 * e + lane;
+        uint32_t kk = 0;
+        if (j < n)
+            kk = ((ff && j == 0) || (fd && j == i)) ? 0xFFFFFFFFu : float_key(srow[j]);
+        key[e] = kk;
+    }
+    uint32_t kth = 0;
+#pragma unroll 1
+    for (int bit = 31; bit >= 0; --bit) {
+        const uint32_t cand = kth | (1u << bit);
+        unsigned cnt = 0;
+#pragma unroll
+        for (int e = 0; e < PER; ++e)
+            cnt += key[e] >= cand ? 1u : 0u;
+        cnt = __reduce_add_sync(0xffffffffu, cnt);
+        if (cnt >= (unsigned)k)
+            kth = cand;
+    }
+    unsigned gt = 0;
+#pragma unroll
+    for (int e = 0; e < PER; ++e)
+        gt += key[e] > kth ? 1u : 0u;
+    gt = __reduce_add_sync(0xffffffffu, gt);
+    const int need_eq = k - (int)gt;
+    int taken = 0;
+#pragma unroll
+    for (int e = 0; e < PER; ++e) {
+        const int j = 32 * e + lane;
+        const bool eq = key[e] == kth && j < n;
+        const uint32_t bal = __ballot_sync(0xffffffffu, eq);
+        const int rank = taken + __popc(bal & ((1u << lane) - 1u));
+        taken += __popc(bal);
+        const bool sel = (j < n) && (key[e] > kth || (eq && rank < need_eq));
+        if (j < nb)
+            mrow[j] = sel ? 1 : 0;
+    }
+    for (int j = 32 * PER + lane; j < nb; j += 32)
+        mrow[j] = 0;
+}
+
 // One warp per row: ascending list of active blocks j <= i and its length.
 __global__ void __launch_bounds__(256)
     compact_kernel(const uint8_t *__restrict__ mask, long long rows, int nb, long long tri, int32_t *__restrict__ lists,
@@ -215,6 +303,18 @@ cudaError_t launch_mask(int B, int Hq, int nb, const float *scores, int mode, fl
         if (blocks > 148LL * 64)
             blocks = 148LL * 64;
         threshold_kernel<<<(unsigned)blocks, kThrThreads, 0, stream>>>(scores, total, nb, threshold, ff, fd, mask);
+        return cudaGetLastError();
+    }
+    if (nb <= 1024) {
+        const unsigned grid = (unsigned)((rows + 7) / 8);
+        if (nb <= 128)
+            topk_warp_kernel<4><<<grid, 256, 0, stream>>>(scores, rows, nb, density, k_fixed, k_per_row, ff, fd, mask);
+        else if (nb <= 256)
+            topk_warp_kernel<8><<<grid, 256, 0, stream>>>(scores, rows, nb, density, k_fixed, k_per_row, ff, fd, mask);
+        else if (nb <= 512)
+            topk_warp_kernel<16><<<grid, 256, 0, stream>>>(scores, rows, nb, density, k_fixed, k_per_row, ff, fd, mask);
+        else
+            topk_warp_kernel<32><<<grid, 256, 0, stream>>>(scores, rows, nb, density, k_fixed, k_per_row, ff, fd, mask);
         return cudaGetLastError();
     }
     const size_t smem = sizeof(uint32_t) * (size_t)nb;

@@ -229,7 +229,8 @@ def _scores_with_ties(B, H, nb, seed):
 
 
 @pytest.mark.parametrize("nb,density,ff,fd", [(40, 0.3, True, True), (257, 0.1, True, True),
-                                              (64, 0.5, False, False), (33, 0.0, True, True)])
+                                              (64, 0.5, False, False), (33, 0.0, True, True),
+                                              (700, 0.2, True, True), (1100, 0.05, False, True)])
 def test_topk_mask_bit_exact(oracle, nb, density, ff, fd):
     s = _scores_with_ties(2, 3, nb, nb)
     m = seer.seer_block_mask(dev(s), "topk", density=density, force_first=ff, force_diag=fd)
