@@ -132,6 +132,24 @@ bool make_tmap_bhsd(CUtensorMap *map, const void *base, int BH, int S, int d)
     return r == CUDA_SUCCESS;
 }
 
+// [B*H, S, d] bf16 viewed as 4-D (64 columns, S rows, d/64 panels, B*H) so
+// that one 64-row box brings every 64-column panel of a block at once,
+// panel-major, each panel in the 128-byte swizzle layout.
+bool make_tmap_bhsd_panels(CUtensorMap *map, const void *base, int BH, int S, int d)
+{
+    EncodeTiledFn fn = encode_fn();
+    if (fn == nullptr)
+        return false;
+    const cuuint64_t dims[4] = {64, (cuuint64_t)S, (cuuint64_t)(d / 64), (cuuint64_t)BH};
+    const cuuint64_t strides[3] = {(cuuint64_t)d * 2, 128, (cuuint64_t)S * d * 2};
+    const cuuint32_t box[4] = {64, 64, (cuuint32_t)(d / 64), 1};
+    const cuuint32_t estr[4] = {1, 1, 1, 1};
+    const CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(base), dims, strides, box,
+                          estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
 } // namespace seer
 
 using namespace seer;

@@ -20,12 +20,14 @@
 //  * S = Q K^T (SS MMA, N = 64) and O += P V (TS MMA: P read from TMEM) with
 //    fp32 accumulators in TMEM: S double-buffered (2 x 64 columns, P aliased
 //    into the first 32 columns of its S buffer), O in 128 columns.
-//  * Warp roles: warps 0-3 softmax / rescale / epilogue (thread = row = TMEM
-//    lane), warp 4 TMA producer, warp 5 MMA issuer + TMEM owner, warp 6 builds
-//    the per-tile active-block list from the mask (the compaction step, fused
-//    here so skipped blocks cost no loads and no extra launch).
-//  * Persistent grid (2 CTAs per SM); tiles are taken heaviest-first (last
-//    query block first) round-robin.
+//  * One CTA per SM (a kernel that allocates TMEM is granted one CTA per SM)
+//    with two independent tile slots.  Per slot: warps 0-3 softmax / rescale /
+//    epilogue (thread = row = TMEM lane), warp 4 TMA producer for Q and K,
+//    warp 5 MMA issuer, warp 6 builds the per-tile active-block list from the
+//    mask (the compaction step, fused so skipped blocks cost no loads and no
+//    extra launch), warp 7 TMA producer for V.
+//  * Persistent grid; tiles are KV-head major (concurrent tiles share one KV
+//    head's K/V in L2), heaviest query blocks first, round-robin.
 //  * The running max is only moved when it grows by more than 2^8 (log2
 //    domain); P = 2^(x - m) then stays <= 256, safe in bf16/fp32, and the O
 //    rescale (TMEM load/store) is rare.
@@ -173,8 +175,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     const int lane = threadIdx.x & 31;
     // Two slots per CTA (one CTA per SM: TMEM allocation pins occupancy to 1).
     // Each slot is an independent tile pipeline: warps 8s+0..3 softmax (TMEM
-    // lane quarters 0..3), 8s+4 TMA producer, 8s+5 MMA issuer, 8s+6 list
-    // builder, 8s+7 spare.  Slot s owns TMEM columns [256 s, 256 s + 256).
+    // lane quarters 0..3), 8s+4 Q/K producer, 8s+5 MMA issuer, 8s+6 list
+    // builder, 8s+7 V producer.  Slot s owns TMEM columns [256 s, 256 s + 256).
     const int slot = warp >> 3;
     const int wl = warp & 7;
     uint8_t *ssm = smem + slot * p.slot_bytes;
@@ -207,7 +209,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                 mbar_init(bi(L::kBarSFull + b), 1);
                 mbar_init(bi(L::kBarPFull + b), kRows);
                 mbar_init(bi(L::kBarListFull + b), 1);
-                mbar_init(bi(L::kBarListEmpty + b), 6);
+                mbar_init(bi(L::kBarListEmpty + b), 7);
             }
             mbar_init(bi(L::kBarODone + 0), 1);
             mbar_init(bi(L::kBarODone + 1), 1);
@@ -309,12 +311,19 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                 mbar_arrive(bar(L::kBarListFull + lb));
             ++n;
         }
-    } else if (wl == 4) {
-        // ------------------------------------------------------------ TMA producer
+    } else if (wl == 4 || wl == 7) {
+        // ------------------------------------------------------------ TMA producers
+        // Warp 4 loads Q and K, warp 7 loads V: a V stage that waits for a late
+        // PV must not hold back the next K tile (S needs K long before PV needs V).
+        const bool kprod = wl == 4;
         if (lane == 0) {
             int n = 0, q_it = 0;
             long long kv_it = 0;
             bool ok = true;
+            const CUtensorMap *tm = kprod ? &tmK : &tmV;
+            const uint32_t sX = kprod ? sK : sV;
+            const int bFull = kprod ? L::kBarKFull : L::kBarVFull;
+            const int bEmpty = kprod ? L::kBarKEmpty : L::kBarVEmpty;
             for (long long u = vcta; u < p.n_units && ok; u += stride) {
                 const Unit un = decode_unit(p, u);
                 if (!un.valid)
@@ -327,52 +336,39 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                 const UnitInfo inf = infos[lb];
                 const uint16_t *lst = lists + lb * list_stride;
                 if (inf.count > 0) {
-                    if (q_it >= 1 && !mbar_wait(bar(L::kBarQEmpty), (q_it - 1) & 1, wc)) {
-                        ok = false;
-                        break;
-                    }
-                    const int halves = inf.h1 >= 0 ? 2 : 1;
-                    mbar_arrive_expect_tx(bar(L::kBarQFull), (uint32_t)(halves * 64 * D * 2));
-                    for (int hf = 0; hf < halves; ++hf) {
-                        const int h = hf ? inf.h1 : inf.h0;
-                        const int i = hf ? inf.i1 : inf.i0;
+                    if (kprod) {
+                        if (q_it >= 1 && !mbar_wait(bar(L::kBarQEmpty), (q_it - 1) & 1, wc)) {
+                            ok = false;
+                            break;
+                        }
+                        const int halves = inf.h1 >= 0 ? 2 : 1;
+                        mbar_arrive_expect_tx(bar(L::kBarQFull), (uint32_t)(halves * 64 * D * 2));
+                        for (int hf = 0; hf < halves; ++hf) {
+                            const int h = hf ? inf.h1 : inf.h0;
+                            const int i = hf ? inf.i1 : inf.i0;
 #pragma unroll
-                        for (int pn = 0; pn < L::kPanels; ++pn)
-                            tma_load_3d(sQ + pn * L::kQPanelBytes + hf * 8192, &tmQ, bar(L::kBarQFull), pn * 64,
-                                        i * 64, inf.b * p.Hq + h);
+                            for (int pn = 0; pn < L::kPanels; ++pn)
+                                tma_load_3d(sQ + pn * L::kQPanelBytes + hf * 8192, &tmQ, bar(L::kBarQFull), pn * 64,
+                                            i * 64, inf.b * p.Hq + h);
+                        }
+                        ++q_it;
                     }
-                    ++q_it;
                     const int zkv = inf.b * p.Hkv + inf.h0 / p.g;
                     for (int t = 0; t < inf.count; ++t) {
                         const int j = lst[t] & 0x3FFF;
                         const int s = (int)(kv_it % kNStage);
                         const long long use = kv_it / kNStage;
-                        if (use >= 1 && !mbar_wait(bar(L::kBarKEmpty + s), (uint32_t)((use - 1) & 1), wc)) {
+                        if (use >= 1 && !mbar_wait(bar(bEmpty + s), (uint32_t)((use - 1) & 1), wc)) {
                             ok = false;
                             break;
                         }
-                        mbar_arrive_expect_tx(bar(L::kBarKFull + s), (uint32_t)(64 * D * 2));
-#pragma unroll
-                        for (int pn = 0; pn < L::kPanels; ++pn)
-                            tma_load_3d(sK + s * L::kKVBytes + pn * L::kKVPanelBytes, &tmK, bar(L::kBarKFull + s),
-                                        pn * 64, j * 64, zkv);
-                        if (use >= 1 && !mbar_wait(bar(L::kBarVEmpty + s), (uint32_t)((use - 1) & 1), wc)) {
-                            ok = false;
-                            break;
-                        }
-                        mbar_arrive_expect_tx(bar(L::kBarVFull + s), (uint32_t)(64 * D * 2));
-#pragma unroll
-                        for (int pn = 0; pn < L::kPanels; ++pn)
-                            tma_load_3d(sV + s * L::kKVBytes + pn * L::kKVPanelBytes, &tmV, bar(L::kBarVFull + s),
-                                        pn * 64, j * 64, zkv);
+                        // One box: 64 keys x all d/64 panels (panel-major, 8 KB per panel).
+                        mbar_arrive_expect_tx(bar(bFull + s), (uint32_t)(64 * D * 2));
+                        tma_load_4d(sX + s * L::kKVBytes, tm, bar(bFull + s), 0, j * 64, 0, zkv);
                         // Warm L2 with the block kPrefetch positions ahead.
                         if (t + kPrefetch < inf.count) {
                             const int jp = lst[t + kPrefetch] & 0x3FFF;
-#pragma unroll
-                            for (int pn = 0; pn < L::kPanels; ++pn) {
-                                tma_prefetch_3d(&tmK, pn * 64, jp * 64, zkv);
-                                tma_prefetch_3d(&tmV, pn * 64, jp * 64, zkv);
-                            }
+                            tma_prefetch_4d(tm, 0, jp * 64, 0, zkv);
                         }
                         ++kv_it;
                     }
@@ -387,12 +383,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                 for (int s = 0; s < kNStage; ++s) {
                     if (kv_it > s) {
                         const long long last = ((kv_it - 1 - s) / kNStage) * kNStage + s;
-                        const uint32_t par = (uint32_t)((last / kNStage) & 1);
-                        mbar_drain(bar(L::kBarKFull + s), par, kDrainNs);
-                        mbar_drain(bar(L::kBarVFull + s), par, kDrainNs);
+                        mbar_drain(bar(bFull + s), (uint32_t)((last / kNStage) & 1), kDrainNs);
                     }
                 }
-                if (q_it > 0)
+                if (kprod && q_it > 0)
                     mbar_drain(bar(L::kBarQFull), (q_it - 1) & 1, kDrainNs);
             }
         }
@@ -698,8 +692,8 @@ template <int D, bool MAP>
 cudaError_t launch_t(const AttnLaunch &a, cudaStream_t stream)
 {
     CUtensorMap tq, tk, tv;
-    if (!make_tmap_bhsd(&tq, a.q, a.B * a.Hq, a.S, D) || !make_tmap_bhsd(&tk, a.k, a.B * a.Hkv, a.S, D) ||
-        !make_tmap_bhsd(&tv, a.v, a.B * a.Hkv, a.S, D))
+    if (!make_tmap_bhsd(&tq, a.q, a.B * a.Hq, a.S, D) || !make_tmap_bhsd_panels(&tk, a.k, a.B * a.Hkv, a.S, D) ||
+        !make_tmap_bhsd_panels(&tv, a.v, a.B * a.Hkv, a.S, D))
         return cudaErrorInvalidValue;
     KParams p;
     p.B = a.B;

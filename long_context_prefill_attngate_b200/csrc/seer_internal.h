@@ -13,7 +13,7 @@ namespace seer {
 constexpr int kBlock = 64;            // block size of gate, mask and kernels
 constexpr int kMaxNb = 16384;         // S <= 1M tokens
 constexpr int kMaxAttnCtas = 296;     // tile pipelines in flight: 2 slots x 148 SMs
-constexpr int kAttnThreads = 512;     // 2 slots x (4 softmax + TMA + MMA + list builder + spare) warps
+constexpr int kAttnThreads = 512;     // 2 slots x (4 softmax + Q/K producer + MMA + list builder + V producer) warps
 
 struct AttnLaunch {
     int B, Hq, Hkv, S, d, nb;
@@ -51,5 +51,6 @@ seer_status set_last_error(seer_status s, const char *fmt, ...);
 
 // Tensor-map creation through the driver entry point (seer_api.cu).
 bool make_tmap_bhsd(CUtensorMap *map, const void *base, int BH, int S, int d);
+bool make_tmap_bhsd_panels(CUtensorMap *map, const void *base, int BH, int S, int d);
 
 } // namespace seer
