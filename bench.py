@@ -63,14 +63,21 @@ def profile_traffic(kernel_src: str, summary: str):
 
 
 class ClockSampler:
-    """nvidia-smi clocks / throttle reasons sampled every 200 ms while running."""
+    """nvidia-smi clocks / throttle reasons sampled every 100 ms while running."""
 
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
     def __init__(self, gpu_index: int):
-        self.gpu = gpu_index
+        # nvidia-smi numbers GPUs physically; identify ours by UUID.
+        self.gpu = str(gpu_index)
+        try:
+            import torch
+            uuid = str(torch.cuda.get_device_properties(gpu_index).uuid)
+            self.gpu = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
+        except Exception:
+            pass
         self.proc = None
         self.path = os.path.join("/tmp", f"seer_clocks_{os.getpid()}.csv")
 
@@ -78,7 +85,7 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "200"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+                 "-lms", "100"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
         except (OSError, FileNotFoundError):
             self.proc = None
         return self
@@ -207,11 +214,16 @@ def run_gpu(args, world, rank, local):
         step = [e[0].elapsed_time(e[3]) for e in ev]
         return dict(gate=gate, mask=msk, attn=att, step=step)
 
-    # ---------------- headline: density from args (default 0.1), timed K steps
+    # ---------------- headline: density from args (default 0.1), timed K steps.
+    # The clock sampler runs through the headline steps and a repeat of them
+    # (same work) so that the sub-second timed region still gets several samples.
     with ClockSampler(local) as clk:
         t_wall0 = time.time()
         res = timed_steps(args.density, args.steps, args.warmup)
         t_wall = time.time() - t_wall0
+        t_end = time.time() + 1.5
+        while time.time() < t_end:
+            timed_steps(args.density, args.steps, 0)
     clocks = clk.summary()
     mask_sum = int(mask.sum(dtype=torch.int64).item())
     flops = attn_flops(mask_sum, w.d)
