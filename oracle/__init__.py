@@ -60,6 +60,7 @@ def _load():
             lib.oracle_compact.argtypes = [P, I, I, I, P, P]
             lib.oracle_masked_attention.argtypes = [P, P, P, I, I, I, I, I, P, D, P, I, P, P]
             lib.oracle_pooled_map.argtypes = [P, P, P, I, I, I, I, I, D, P, I, P, P]
+            lib.oracle_distill_loss.argtypes = [P, P, I, I, I, P, P, P]
             _lib = lib
     return _lib
 
@@ -230,3 +231,17 @@ def pooled_map(q, k, v, scale: float | None = None, units=None):
     _load().oracle_pooled_map(_ptr(q), _ptr(k), _ptr(v), B, Hq, Hkv, S, d, float(scale),
                               _ptr(units), n, _ptr(o), _ptr(A))
     return o, A
+
+
+def distill_loss(G, A):
+    """Row-normalised target Ahat, per-row squared error and per-head mean
+    (over causal block entries) of MSE(G, Ahat); G, A f32 [B,Hq,nb,nb]."""
+    G = np.ascontiguousarray(G, dtype=np.float32)
+    A = np.ascontiguousarray(A, dtype=np.float32)
+    B, Hq, nb, _ = G.shape
+    assert A.shape == G.shape
+    ahat = np.empty((B, Hq, nb, nb), np.float64)
+    rows = np.empty((B, Hq, nb), np.float64)
+    heads = np.empty((B, Hq), np.float64)
+    _load().oracle_distill_loss(_ptr(G), _ptr(A), B, Hq, nb, _ptr(ahat), _ptr(rows), _ptr(heads))
+    return ahat, rows, heads

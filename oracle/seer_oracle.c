@@ -415,3 +415,47 @@ void oracle_pooled_map(const uint16_t *q, const uint16_t *k, const uint16_t *v,
         free(qrow);
     }
 }
+
+/* ---------------------------------------------------------------------------
+ * Distillation target and loss ["Learning Intrinsic Sparse Attention",
+ * rebuttal Question 2: the max-pooled map is row-normalised so that it matches
+ * the gate's softmax output (row sum 1); Q2 on the loss: the gate is trained
+ * with an MSE loss against that target].
+ * G (gate soft scores) and A (max-pooled map): f32 [B, Hq, nb, nb].
+ *   Ahat[i, j] = A[i, j] / sum_{j' <= i} A[i, j']      (0 for j > i; 0 row stays 0)
+ *   loss_rows[b, h, i] = sum_{j <= i} (G[i, j] - Ahat[i, j])^2
+ *   loss_heads[b, h]   = sum_i loss_rows[b, h, i] / (nb (nb + 1) / 2)
+ * (the mean over the causal block entries: a reading, the pages do not say
+ * which entries the mean runs over).
+ * ------------------------------------------------------------------------- */
+void oracle_distill_loss(const float *G, const float *A, int B, int Hq, int nb, double *Ahat, double *loss_rows,
+                         double *loss_heads)
+{
+    const long long units = (long long)B * Hq * nb;
+#pragma omp parallel for schedule(static)
+    for (long long u = 0; u < units; ++u) {
+        const int i = (int)(u % nb);
+        const float *a = A + u * nb;
+        const float *g = G + u * nb;
+        double *ah = Ahat + u * nb;
+        double sum = 0.0;
+        for (int j = 0; j <= i; ++j)
+            sum += (double)a[j];
+        double l = 0.0;
+        for (int j = 0; j < nb; ++j) {
+            ah[j] = (j <= i && sum > 0.0) ? (double)a[j] / sum : 0.0;
+            if (j <= i) {
+                const double dlt = (double)g[j] - ah[j];
+                l += dlt * dlt;
+            }
+        }
+        loss_rows[u] = l;
+    }
+    const double tri = (double)nb * (nb + 1) / 2.0;
+    for (long long bh = 0; bh < (long long)B * Hq; ++bh) {
+        double s = 0.0;
+        for (int i = 0; i < nb; ++i)
+            s += loss_rows[bh * nb + i];
+        loss_heads[bh] = s / tri;
+    }
+}

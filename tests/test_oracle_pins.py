@@ -378,3 +378,35 @@ def test_pooled_map_units_subset_matches_full(oracle):
         idx = (b * Hq + h) * nb + i
         np.testing.assert_array_equal(o[n], of[idx])
         np.testing.assert_array_equal(A[n], Af[idx])
+
+
+# ------------------------------------------------------------ distillation loss
+def test_distill_loss_pins(oracle):
+    B, Hq, nb = 2, 3, 9
+    r = rng(90)
+    G = np.tril(r.random((B, Hq, nb, nb))).astype(np.float32)
+    G /= G.sum(-1, keepdims=True)
+    G = G.astype(np.float32)
+    # A proportional to G row by row -> target equals G (up to f32 rounding) -> loss ~ 0
+    scale = r.random((B, Hq, nb, 1)).astype(np.float32) + 0.5
+    ahat, rows, heads = oracle.distill_loss(G, (G * scale).astype(np.float32))
+    np.testing.assert_allclose(ahat, G, rtol=1e-6, atol=1e-7)
+    assert np.all(heads < 1e-12)
+    # rows of the target sum to 1; zero rows stay zero; loss is then sum G^2
+    A = np.tril(r.random((B, Hq, nb, nb))).astype(np.float32)
+    A[0, 1, 4, :] = 0
+    ahat, rows, heads = oracle.distill_loss(G, A)
+    s = ahat.sum(-1)
+    s[0, 1, 4] = 1.0
+    np.testing.assert_allclose(s, 1.0, rtol=1e-12)
+    assert np.all(ahat[0, 1, 4] == 0)
+    np.testing.assert_allclose(rows[0, 1, 4], (G[0, 1, 4].astype(np.float64) ** 2).sum(), rtol=1e-12)
+    # brute force
+    Ad, Gd = A.astype(np.float64), G.astype(np.float64)
+    tot = Ad.sum(-1, keepdims=True)
+    want_hat = np.where(tot > 0, Ad / np.where(tot > 0, tot, 1), 0.0)
+    np.testing.assert_allclose(ahat, want_hat, rtol=1e-12, atol=0)
+    lower = np.tril(np.ones((nb, nb), bool))
+    want_rows = (((Gd - want_hat) ** 2) * lower).sum(-1)
+    np.testing.assert_allclose(rows, want_rows, rtol=1e-12)
+    np.testing.assert_allclose(heads, want_rows.sum(-1) / (nb * (nb + 1) / 2), rtol=1e-12)
