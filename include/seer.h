@@ -192,6 +192,21 @@ SEER_API seer_status seer_gate_scores_noalloc(const seer_shape *shape, const voi
                                               const void *wq, const void *wk, const seer_gate_params *gp,
                                               float *scores, void *stream);
 
+/*
+ * seer_distill_loss — the gate's distillation target and MSE loss
+ * ("Learning Intrinsic Sparse Attention", rebuttal Question 2: the max-pooled
+ * map is row-normalised to match the gate's softmax output; Q2 on the loss:
+ * MSE against that target).  For soft scores G = scores and pooled map A
+ * (fp32 [B,Hq,nb,nb], e.g. from seer_gate_scores and seer_attn_pooled_map):
+ *   A_norm[i,j]     = A[i,j] / sum_{j'<=i} A[i,j']  (0 for j > i; zero rows stay 0)
+ *   loss_rows[b,h,i] = sum_{j<=i} (G[i,j] - A_norm[i,j])^2        fp32 [B,Hq,nb]
+ *   loss[b,h]       = sum_i loss_rows[b,h,i] / (nb(nb+1)/2)        fp32 [B,Hq]
+ * (mean over the causal block entries).  A_norm may be NULL (not written).
+ * Reductions run in a fixed order: results are reproducible.  No workspace.
+ */
+SEER_API seer_status seer_distill_loss(const seer_shape *shape, const float *scores, const float *A,
+                                       float *A_norm, float *loss_rows, float *loss, void *stream);
+
 /* Workspace bytes a call needs for `shape` (0 for SEER_CALL_BLOCK_SPARSE_PREFILL).
  * Returns 0 and sets the last error for an invalid shape or call id. */
 SEER_API size_t seer_workspace_bytes(int which_call, const seer_shape *shape);

@@ -37,7 +37,7 @@ BLOCK = 64
 EXPORTS = (
     "seer_gate_scores", "seer_block_mask", "seer_compact_mask", "seer_block_sparse_prefill",
     "seer_attn_pooled_map", "seer_workspace_bytes", "seer_check_status", "seer_set_wait_timeout_ns",
-    "seer_last_error", "seer_version", "seer_gate_scores_noalloc",
+    "seer_last_error", "seer_version", "seer_gate_scores_noalloc", "seer_distill_loss",
 )
 
 
@@ -83,10 +83,12 @@ def lib() -> ctypes.CDLL:
             L.seer_gate_scores_noalloc.argtypes = [SP, P, P, P, P, ctypes.POINTER(seer_gate_params), P, P]
             L.seer_block_mask.argtypes = [SP, P, ctypes.POINTER(seer_mask_params), P, P]
             L.seer_compact_mask.argtypes = [SP, P, P, P, P]
+            L.seer_distill_loss.argtypes = [SP, P, P, P, P, P, P]
             L.seer_block_sparse_prefill.argtypes = [SP, P, P, P, P, F, P, P, P, Z, P]
             L.seer_attn_pooled_map.argtypes = [SP, P, P, P, F, P, P, P, Z, P]
             for fn in ("seer_gate_scores", "seer_gate_scores_noalloc", "seer_block_mask", "seer_compact_mask",
-                       "seer_block_sparse_prefill", "seer_attn_pooled_map", "seer_check_status"):
+                       "seer_block_sparse_prefill", "seer_attn_pooled_map", "seer_check_status",
+                       "seer_distill_loss"):
                 getattr(L, fn).restype = I
             L.seer_workspace_bytes.argtypes = [I, SP]
             L.seer_workspace_bytes.restype = Z
@@ -270,6 +272,24 @@ def seer_attn_pooled_map(q, k, v, softmax_scale: float = 0.0, o=None, A=None, wo
     _check(lib().seer_attn_pooled_map(ctypes.byref(sh), _ptr(q), _ptr(k), _ptr(v), float(softmax_scale), _ptr(o),
                                       _ptr(A), _ptr(workspace), wsb, _stream_ptr(stream)))
     return o, A
+
+
+def seer_distill_loss(scores, A, want_norm: bool = False, stream=None, Hkv: int = 1, d: int = 64):
+    """Row-normalised target, per-row squared error and per-head MSE (see include/seer.h).
+
+    Returns (loss [B,Hq], loss_rows [B,Hq,nb], A_norm or None)."""
+    torch = _torch()
+    _need(scores.dtype == A.dtype == torch.float32 and scores.is_contiguous() and A.is_contiguous(),
+          "scores and A must be contiguous fp32")
+    _need(scores.shape == A.shape, "scores and A must have the same shape")
+    B, Hq, nb, _ = scores.shape
+    sh = seer_shape(B, Hq, Hkv if Hq % Hkv == 0 else 1, nb * BLOCK, d)
+    rows = torch.empty((B, Hq, nb), dtype=torch.float32, device=scores.device)
+    loss = torch.empty((B, Hq), dtype=torch.float32, device=scores.device)
+    an = torch.empty_like(A) if want_norm else None
+    _check(lib().seer_distill_loss(ctypes.byref(sh), _ptr(scores), _ptr(A), _ptr(an), _ptr(rows), _ptr(loss),
+                                   _stream_ptr(stream)))
+    return loss, rows, an
 
 
 def topk_counts(density: float, nb: int, force_first: bool = True, force_diag: bool = True) -> list[int]:

@@ -350,6 +350,21 @@ seer_status seer_attn_pooled_map(const seer_shape *shape, const void *q, const v
     return ok();
 }
 
+seer_status seer_distill_loss(const seer_shape *shape, const float *scores, const float *A, float *A_norm,
+                              float *loss_rows, float *loss, void *stream)
+{
+    seer_status st = check_shape(shape);
+    if (st != SEER_OK)
+        return st;
+    if (scores == nullptr || A == nullptr || loss_rows == nullptr || loss == nullptr)
+        return fail(SEER_ERR_INVALID_ARG, "seer_distill_loss: NULL scores, A, loss_rows or loss");
+    const cudaError_t e = launch_distill(shape->B, shape->Hq, shape->S / kBlock, scores, A, A_norm, loss_rows, loss,
+                                         static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess)
+        return cuda_fail(e, "seer_distill_loss launch");
+    return ok();
+}
+
 seer_status seer_check_status(void *stream)
 {
     cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));

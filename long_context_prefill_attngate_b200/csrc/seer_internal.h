@@ -46,6 +46,10 @@ cudaError_t launch_mask(int B, int Hq, int nb, const float *scores, int mode, fl
 cudaError_t launch_compact(int B, int Hq, int nb, const uint8_t *mask, int32_t *lists, int32_t *counts,
                            cudaStream_t stream);
 
+// Distillation target and loss (seer_distill.cu).
+cudaError_t launch_distill(int B, int Hq, int nb, const float *G, const float *A, float *ahat, float *loss_rows,
+                           float *loss, cudaStream_t stream);
+
 // Record the thread-local error text returned by seer_last_error() (seer_api.cu).
 seer_status set_last_error(seer_status s, const char *fmt, ...);
 

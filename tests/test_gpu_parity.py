@@ -360,3 +360,31 @@ def test_prefill_repeated_calls_block_attribution(oracle):
         o = seer.seer_block_sparse_prefill(q, k, vd, md)
         seer.seer_check_status()
         check_o(o.cpu().reshape(-1, BLOCK, d), o_ref, "O(one-hot V)")
+
+
+# ------------------------------------------------------------------ distillation target and loss
+@pytest.mark.parametrize("name", ["tiny", "map"])
+def test_distill_loss(oracle, name):
+    if name == "tiny":
+        w = syn.WORKLOADS["tiny"]
+    else:
+        w = syn.custom("distill", 1, 5, 1, 2048, 128, number=81)
+    x = syn.make_inputs(w)
+    q, k, v = dev(x["q"]), dev(x["k"]), dev(x["v"])
+    G = seer.seer_gate_scores(q, k, dev(x["wq"]), dev(x["wk"]), rope_theta=w.rope_theta)
+    _, A = seer.seer_attn_pooled_map(q, k, v)
+    loss, rows, an = seer.seer_distill_loss(G, A, want_norm=True, Hkv=w.Hkv, d=w.d)
+    seer.seer_check_status()
+    ahat_ref, rows_ref, heads_ref = oracle.distill_loss(G.cpu().numpy(), A.cpu().numpy())
+    check_rel(an.cpu().numpy(), ahat_ref, "A_norm")
+    check_rel(rows.cpu().numpy(), rows_ref, "loss rows")
+    check_rel(loss.cpu().numpy(), heads_ref, "loss")
+    # reproducible
+    loss2, _, _ = seer.seer_distill_loss(G, A, Hkv=w.Hkv, d=w.d)
+    assert torch.equal(loss, loss2)
+    # and the whole chain against the oracle's own gate and map (fp64)
+    if name == "tiny":
+        Go = oracle.gate_scores(bits(x["q"]), bits(x["k"]), bits(x["wq"]), bits(x["wk"]), theta=w.rope_theta)
+        _, Ao = oracle.pooled_map(bits(x["q"]), bits(x["k"]), bits(x["v"]))
+        _, _, heads_o = oracle.distill_loss(Go.astype(np.float32), Ao.reshape(Go.shape).astype(np.float32))
+        check_rel(loss.cpu().numpy(), heads_o, "loss (oracle chain)")
