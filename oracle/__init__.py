@@ -61,6 +61,8 @@ def _load():
             lib.oracle_masked_attention.argtypes = [P, P, P, I, I, I, I, I, P, D, P, I, P, P]
             lib.oracle_pooled_map.argtypes = [P, P, P, I, I, I, I, I, D, P, I, P, P]
             lib.oracle_distill_loss.argtypes = [P, P, I, I, I, P, P, P]
+            lib.oracle_pool_maxmin.argtypes = [P, I, I, I, I, P]
+            lib.oracle_gate_scores_kpool.argtypes = [P, P, I, I, I, I, I, P, LL, P, LL, I, D, I, P]
             _lib = lib
     return _lib
 
@@ -88,6 +90,15 @@ def pool_avg(x: np.ndarray) -> np.ndarray:
     B, H, S, d = x.shape
     out = np.empty((B, H, S // BLOCK, d), np.float64)
     _load().oracle_pool_avg(_ptr(x), B, H, S, d, _ptr(out))
+    return out
+
+
+def pool_maxmin(x: np.ndarray) -> np.ndarray:
+    """a1': per-block max and min, concatenated; bf16 [B,H,S,d] -> f64 [B,H,S/64,2d]."""
+    x = _u16(x)
+    B, H, S, d = x.shape
+    out = np.empty((B, H, S // BLOCK, 2 * d), np.float64)
+    _load().oracle_pool_maxmin(_ptr(x), B, H, S, d, _ptr(out))
     return out
 
 
@@ -122,20 +133,23 @@ def block_softmax(qt: np.ndarray, kt: np.ndarray) -> np.ndarray:
     return out
 
 
-def gate_scores(q, k, wq, wk, theta: float = 5e5, wq_head_stride=None, wk_head_stride=None) -> np.ndarray:
-    """a1-a3: AttnGate soft scores, f64 [B,Hq,nb,nb]."""
+def gate_scores(q, k, wq, wk, theta: float = 5e5, wq_head_stride=None, wk_head_stride=None,
+                k_maxmin: bool = False) -> np.ndarray:
+    """a1-a3: AttnGate soft scores, f64 [B,Hq,nb,nb].  With k_maxmin, K is
+    pooled by [max | min] and wk is [Hkv, 2d, dg]."""
     q, k, wq, wk = _u16(q), _u16(k), _u16(wq), _u16(wk)
     B, Hq, S, d = q.shape
     Hkv = k.shape[1]
     dg = wq.shape[-1]
+    dk = 2 * d if k_maxmin else d
     if wq_head_stride is None:
         wq_head_stride = 0 if wq.ndim == 2 else d * dg
     if wk_head_stride is None:
-        wk_head_stride = 0 if wk.ndim == 2 else d * dg
+        wk_head_stride = 0 if wk.ndim == 2 else dk * dg
     nb = S // BLOCK
     out = np.empty((B, Hq, nb, nb), np.float64)
-    _load().oracle_gate_scores(_ptr(q), _ptr(k), B, Hq, Hkv, S, d, _ptr(wq), int(wq_head_stride),
-                               _ptr(wk), int(wk_head_stride), dg, float(theta), _ptr(out))
+    _load().oracle_gate_scores_kpool(_ptr(q), _ptr(k), B, Hq, Hkv, S, d, _ptr(wq), int(wq_head_stride),
+                                     _ptr(wk), int(wk_head_stride), dg, float(theta), int(bool(k_maxmin)), _ptr(out))
     return out
 
 

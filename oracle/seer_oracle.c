@@ -81,6 +81,39 @@ void oracle_pool_avg(const uint16_t *x, int B, int H, int S, int d, double *out)
 }
 
 /* ---------------------------------------------------------------------------
+ * a1' [GATE Weakness 3: "Max+Min pooling in K ... concated in hidden dim
+ * before the linear layer ([Batch, Head, Seq / Block, Dim * 2])"; Question 1:
+ * K prefers max-min pooling]:
+ * out[b,h,i,c]     = max_{t<64} x[b,h,64 i + t, c]
+ * out[b,h,i,d + c] = min_{t<64} x[b,h,64 i + t, c]      (max first: a reading)
+ * x: bf16 [B, H, S, d]  ->  out: f64 [B, H, S/64, 2d]
+ * ------------------------------------------------------------------------- */
+void oracle_pool_maxmin(const uint16_t *x, int B, int H, int S, int d, double *out)
+{
+    const int nb = S / SEER_ORACLE_BLOCK;
+    const long long units = (long long)B * H * nb;
+#pragma omp parallel for schedule(static)
+    for (long long u = 0; u < units; ++u) {
+        const long long bh = u / nb;
+        const int i = (int)(u % nb);
+        const uint16_t *base = x + (bh * S + (long long)i * SEER_ORACLE_BLOCK) * d;
+        double *o = out + u * 2 * d;
+        for (int c = 0; c < d; ++c) {
+            double mx = -INFINITY, mn = INFINITY;
+            for (int t = 0; t < SEER_ORACLE_BLOCK; ++t) {
+                const double v = bf16_to_f64(base[(long long)t * d + c]);
+                if (v > mx)
+                    mx = v;
+                if (v < mn)
+                    mn = v;
+            }
+            o[c] = mx;
+            o[d + c] = mn;
+        }
+    }
+}
+
+/* ---------------------------------------------------------------------------
  * Block RoPE [GATE Q1 on AttnGate's RoPE]: rotate-half pairs (t, t + dg/2)
  * by angle p * theta^(-2t/dg), p = block index.  In place on one vector.
  * ------------------------------------------------------------------------- */
@@ -165,26 +198,40 @@ void oracle_block_softmax(const double *qt, const double *kt, int B, int Hq,
     }
 }
 
+void oracle_gate_scores_kpool(const uint16_t *q, const uint16_t *k, int B, int Hq,
+                              int Hkv, int S, int d, const uint16_t *wq,
+                              long long wq_head_stride, const uint16_t *wk,
+                              long long wk_head_stride, int dg, double theta,
+                              int k_maxmin, double *scores)
+{
+    const int nb = S / SEER_ORACLE_BLOCK;
+    const int dk = k_maxmin ? 2 * d : d;
+    double *qp = (double *)malloc(sizeof(double) * (size_t)B * Hq * nb * d);
+    double *kp = (double *)malloc(sizeof(double) * (size_t)B * Hkv * nb * dk);
+    double *qt = (double *)malloc(sizeof(double) * (size_t)B * Hq * nb * dg);
+    double *kt = (double *)malloc(sizeof(double) * (size_t)B * Hkv * nb * dg);
+    oracle_pool_avg(q, B, Hq, S, d, qp);
+    if (k_maxmin)
+        oracle_pool_maxmin(k, B, Hkv, S, d, kp);
+    else
+        oracle_pool_avg(k, B, Hkv, S, d, kp);
+    oracle_project_rope(qp, B, Hq, nb, d, wq, wq_head_stride, dg, theta, qt);
+    oracle_project_rope(kp, B, Hkv, nb, dk, wk, wk_head_stride, dg, theta, kt);
+    oracle_block_softmax(qt, kt, B, Hq, Hkv, nb, dg, scores);
+    free(qp);
+    free(kp);
+    free(qt);
+    free(kt);
+}
+
 void oracle_gate_scores(const uint16_t *q, const uint16_t *k, int B, int Hq,
                         int Hkv, int S, int d, const uint16_t *wq,
                         long long wq_head_stride, const uint16_t *wk,
                         long long wk_head_stride, int dg, double theta,
                         double *scores)
 {
-    const int nb = S / SEER_ORACLE_BLOCK;
-    double *qp = (double *)malloc(sizeof(double) * (size_t)B * Hq * nb * d);
-    double *kp = (double *)malloc(sizeof(double) * (size_t)B * Hkv * nb * d);
-    double *qt = (double *)malloc(sizeof(double) * (size_t)B * Hq * nb * dg);
-    double *kt = (double *)malloc(sizeof(double) * (size_t)B * Hkv * nb * dg);
-    oracle_pool_avg(q, B, Hq, S, d, qp);
-    oracle_pool_avg(k, B, Hkv, S, d, kp);
-    oracle_project_rope(qp, B, Hq, nb, d, wq, wq_head_stride, dg, theta, qt);
-    oracle_project_rope(kp, B, Hkv, nb, d, wk, wk_head_stride, dg, theta, kt);
-    oracle_block_softmax(qt, kt, B, Hq, Hkv, nb, dg, scores);
-    free(qp);
-    free(kp);
-    free(qt);
-    free(kt);
+    oracle_gate_scores_kpool(q, k, B, Hq, Hkv, S, d, wq, wq_head_stride, wk, wk_head_stride, dg, theta, 0,
+                             scores);
 }
 
 /* ---------------------------------------------------------------------------

@@ -410,3 +410,44 @@ def test_distill_loss_pins(oracle):
     want_rows = (((Gd - want_hat) ** 2) * lower).sum(-1)
     np.testing.assert_allclose(rows, want_rows, rtol=1e-12)
     np.testing.assert_allclose(heads, want_rows.sum(-1) / (nb * (nb + 1) / 2), rtol=1e-12)
+
+
+# ------------------------------------------------------------ max+min K pooling
+def test_pool_maxmin_pins(oracle):
+    bits = rand_bits((2, 3, 192, 16), 91)
+    x = bits_to_f64(bits).reshape(2, 3, 3, BLOCK, 16)
+    out = oracle.pool_maxmin(bits)
+    np.testing.assert_array_equal(out[..., :16], x.max(axis=3))
+    np.testing.assert_array_equal(out[..., 16:], x.min(axis=3))
+    # constant blocks: max == min == the constant
+    const = f64_to_bits(np.full((1, 1, 128, 4), 0.75))
+    o = oracle.pool_maxmin(const)
+    assert np.all(o == 0.75)
+
+
+def test_gate_scores_maxmin_brute_force(oracle):
+    B, Hq, Hkv, S, d, dg = 1, 4, 2, 512, 16, 8
+    qb, kb = rand_bits((B, Hq, S, d), 92, scale=3.0), rand_bits((B, Hkv, S, d), 93, scale=3.0)
+    wqb, wkb = rand_bits((Hq, d, dg), 94, scale=0.5), rand_bits((Hkv, 2 * d, dg), 95, scale=0.5)
+    got = oracle.gate_scores(qb, kb, wqb, wkb, theta=1e2, k_maxmin=True)
+    q, k = bits_to_f64(qb), bits_to_f64(kb)
+    nb = S // BLOCK
+    qp = q.reshape(B, Hq, nb, BLOCK, d).mean(3)
+    kr = k.reshape(B, Hkv, nb, BLOCK, d)
+    kp = np.concatenate([kr.max(3), kr.min(3)], -1)
+    qt = np.einsum("bhid,hde->bhie", qp, bits_to_f64(wqb))
+    kt = np.einsum("bhid,hde->bhie", kp, bits_to_f64(wkb))
+    rot = np.exp(1j * np.arange(nb)[:, None] * 1e2 ** (-2.0 * np.arange(dg // 2) / dg)[None, :])
+
+    def apply(xx):
+        z = (xx[..., : dg // 2] + 1j * xx[..., dg // 2:]) * rot
+        return np.concatenate([z.real, z.imag], -1)
+
+    qt, kt = apply(qt), np.repeat(apply(kt), Hq // Hkv, axis=1)
+    lg = np.einsum("bhie,bhje->bhij", qt, kt) / math.sqrt(dg)
+    lg = np.where(np.tril(np.ones((nb, nb), bool)), lg, -np.inf)
+    e = np.exp(lg - lg.max(-1, keepdims=True))
+    np.testing.assert_allclose(got, e / e.sum(-1, keepdims=True), rtol=1e-11, atol=1e-15)
+    # the avg path is unchanged by the new entry point
+    np.testing.assert_array_equal(oracle.gate_scores(qb, kb, wqb, rand_bits((Hkv, d, dg), 96)),
+                                  oracle.gate_scores(qb, kb, wqb, rand_bits((Hkv, d, dg), 96), k_maxmin=False))
