@@ -279,6 +279,24 @@ def run_gpu(args, world, rank, local):
         ms = statistics.median(ts)
         pooled = {"ms": round(ms, 3), "active_tflops": round(fl / (ms * 1e-3) / 1e12, 1),
                   "frac_of_bf16_peak": round(fl / (ms * 1e-3) / 1e12 / pk["bf16_tflops"], 4)}
+        # Distillation loss on the same layer: gate scores vs the row-normalised map.
+        seer.seer_gate_scores(q, k, wq, wk, rope_theta=w.rope_theta, scores=scores, workspace=gws)
+        for _ in range(3):
+            seer.seer_distill_loss(scores, A, Hkv=w.Hkv, d=w.d)
+        ts = []
+        for _ in range(5):
+            flush.zero_()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            seer.seer_distill_loss(scores, A, Hkv=w.Hkv, d=w.d)
+            e1.record(stream)
+            torch.cuda.synchronize()
+            ts.append(e0.elapsed_time(e1))
+        seer.seer_check_status()
+        ms = statistics.median(ts)
+        byt = 2 * 4 * w.B * w.Hq * nb * nb + 4 * w.B * w.Hq * nb
+        pooled["distill_loss"] = {"ms": round(ms, 4), "gbs": round(byt / (ms * 1e-3) / 1e9, 1),
+                                  "frac_of_hbm_peak": round(byt / (ms * 1e-3) / 1e9 / pk["hbm_gbs"], 4)}
         del A, mws, om
 
     # ---------------- e2e: pinned host inputs -> C ABI -> host output, per step
@@ -321,6 +339,10 @@ def run_gpu(args, world, rank, local):
 
     traffic = profile_traffic("long_context_prefill_attngate_b200/csrc/seer_attn.cu",
                               "attn_sparse_llama8b_32k_d0.1.md")
+    # Algorithmic bytes: gate reads Q and K once and writes the scores; the
+    # mask reads the causal scores and writes the mask.
+    gate_bytes = 2 * (w.B * w.Hq * w.S * w.d + w.B * w.Hkv * w.S * w.d) + 4 * w.B * w.Hq * nb * nb
+    mask_bytes = 4 * w.B * w.Hq * nb * (nb + 1) // 2 + w.B * w.Hq * nb * nb
     launches_per_step = 5 + 1 + 1   # gate: 2 pool + 2 project/RoPE + 1 softmax; mask: 1; attention: 1
     out = {
         "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world, "steps": args.steps,
@@ -332,6 +354,10 @@ def run_gpu(args, world, rank, local):
                    "l2": "flushed between timed steps (256 MiB write, outside the step events)",
                    "parallelism": "replicas" if world > 1 else "single"},
         "ms_layer_attention": round(ms_attn, 4), "ms_gate": round(ms_gate, 4), "ms_mask": round(ms_mask, 4),
+        "gate_hbm": {"algorithmic_bytes": gate_bytes, "gbs": round(gate_bytes / (ms_gate * 1e-3) / 1e9, 1),
+                     "frac_of_hbm_peak": round(gate_bytes / (ms_gate * 1e-3) / 1e9 / pk["hbm_gbs"], 4)},
+        "mask_hbm": {"algorithmic_bytes": mask_bytes, "gbs": round(mask_bytes / (ms_mask * 1e-3) / 1e9, 1),
+                     "frac_of_hbm_peak": round(mask_bytes / (ms_mask * 1e-3) / 1e9 / pk["hbm_gbs"], 4)},
         "attention_active_tflops": round(attn_tflops, 1),
         "roofline": {"bound": "tensor", "achieved": round(attn_tflops, 1), "peak": pk["bf16_tflops"],
                      "unit": "TFLOP/s", "frac": round(attn_tflops / pk["bf16_tflops"], 4), "traffic": traffic,

@@ -75,7 +75,14 @@ typedef struct seer_gate_params {
     float rope_theta;
     long long wq_head_stride;
     long long wk_head_stride;
+    int k_pooling;            /* SEER_KPOOL_AVG (0) or SEER_KPOOL_MAXMIN (1)          */
 } seer_gate_params;
+
+/* K pooling of the gate ("Learning Intrinsic Sparse Attention", rebuttal
+ * Weakness 3 and Question 1): average like Q, or per-block max and min
+ * concatenated along the feature axis ([max | min], 2d features; W_k is then
+ * bf16 [2d, d_gate] per KV head). */
+enum { SEER_KPOOL_AVG = 0, SEER_KPOOL_MAXMIN = 1 };
 
 /* Mask modes ("SeerAttention-Llama-3.1-8B-AttnGates": threshold/TopK on the
  * soft scores; "Learning Intrinsic Sparse Attention", Weakness 2: TopK is
@@ -109,6 +116,8 @@ enum {
  *   Qp = mean over each 64-token block of q   (K likewise: average pooling)
  *   Qt = RoPE_i(Qp @ Wq[h]),  Kt = RoPE_j(Kp @ Wk[h_kv])
  *   scores[b,h,i,j] = softmax_{j<=i}(Qt_i . Kt_j / sqrt(d_gate)); 0 for j > i.
+ * With k_pooling = SEER_KPOOL_MAXMIN, Kp = [max | min] over each block (2d
+ * features) and W_k is [2d, d_gate].
  * q: bf16 [B,Hq,S,d]; k: bf16 [B,Hkv,S,d]; wq/wk: bf16 per the params;
  * scores: fp32 [B,Hq,nb,nb] (fully written).  Workspace:
  * seer_workspace_bytes(SEER_CALL_GATE_SCORES, shape) bytes, 256-B aligned.

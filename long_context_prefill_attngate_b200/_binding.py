@@ -52,9 +52,13 @@ class seer_shape(ctypes.Structure):
                 ("d", ctypes.c_int)]
 
 
+SEER_KPOOL_AVG = 0
+SEER_KPOOL_MAXMIN = 1
+
+
 class seer_gate_params(ctypes.Structure):
     _fields_ = [("d_gate", ctypes.c_int), ("rope_theta", ctypes.c_float), ("wq_head_stride", ctypes.c_longlong),
-                ("wk_head_stride", ctypes.c_longlong)]
+                ("wk_head_stride", ctypes.c_longlong), ("k_pooling", ctypes.c_int)]
 
 
 class seer_mask_params(ctypes.Structure):
@@ -160,7 +164,8 @@ def _workspace(which: int, sh: seer_shape, device, workspace):
 
 
 def seer_gate_scores(q, k, wq, wk, rope_theta: float = 5e5, scores=None, workspace=None, stream=None,
-                     wq_head_stride: int | None = None, wk_head_stride: int | None = None):
+                     wq_head_stride: int | None = None, wk_head_stride: int | None = None,
+                     k_maxmin: bool = False):
     """AttnGate soft scores fp32 [B,Hq,nb,nb] (see include/seer.h)."""
     torch = _torch()
     _need(q.is_contiguous() and k.is_contiguous() and wq.is_contiguous() and wk.is_contiguous(),
@@ -172,18 +177,21 @@ def seer_gate_scores(q, k, wq, wk, rope_theta: float = 5e5, scores=None, workspa
     if wq_head_stride is None:
         wq_head_stride = 0 if wq.dim() == 2 else d * dg
     if wk_head_stride is None:
-        wk_head_stride = 0 if wk.dim() == 2 else d * dg
+        wk_head_stride = 0 if wk.dim() == 2 else (2 * d if k_maxmin else d) * dg
+    _need(wk.shape[-2] == (2 * d if k_maxmin else d) and wk.shape[-1] == dg,
+          "wk must be [.., %d, %d] for %s K pooling" % (2 * d if k_maxmin else d, dg, "max+min" if k_maxmin else "average"))
     if scores is None:
         scores = torch.empty((sh.B, sh.Hq, nb, nb), dtype=torch.float32, device=q.device)
     workspace, wsb = _workspace(SEER_CALL_GATE_SCORES, sh, q.device, workspace)
-    gp = seer_gate_params(int(dg), float(rope_theta), int(wq_head_stride), int(wk_head_stride))
+    gp = seer_gate_params(int(dg), float(rope_theta), int(wq_head_stride), int(wk_head_stride), int(bool(k_maxmin)))
     _check(lib().seer_gate_scores(ctypes.byref(sh), _ptr(q), _ptr(k), _ptr(wq), _ptr(wk), ctypes.byref(gp),
                                   _ptr(scores), _ptr(workspace), wsb, _stream_ptr(stream)))
     return scores
 
 
 def seer_gate_scores_noalloc(q, k, wq, wk, rope_theta: float = 5e5, scores=None, stream=None,
-                             wq_head_stride: int | None = None, wk_head_stride: int | None = None):
+                             wq_head_stride: int | None = None, wk_head_stride: int | None = None,
+                             k_maxmin: bool = False):
     """seer_gate_scores without a workspace: the library's fixed scratch is used
     (for callers that cannot allocate device memory; shapes needing more than
     24 MiB of gate scratch raise SeerError)."""
@@ -196,10 +204,12 @@ def seer_gate_scores_noalloc(q, k, wq, wk, rope_theta: float = 5e5, scores=None,
     if wq_head_stride is None:
         wq_head_stride = 0 if wq.dim() == 2 else d * dg
     if wk_head_stride is None:
-        wk_head_stride = 0 if wk.dim() == 2 else d * dg
+        wk_head_stride = 0 if wk.dim() == 2 else (2 * d if k_maxmin else d) * dg
+    _need(wk.shape[-2] == (2 * d if k_maxmin else d) and wk.shape[-1] == dg,
+          "wk must be [.., %d, %d] for %s K pooling" % (2 * d if k_maxmin else d, dg, "max+min" if k_maxmin else "average"))
     if scores is None:
         scores = torch.empty((sh.B, sh.Hq, nb, nb), dtype=torch.float32, device=q.device)
-    gp = seer_gate_params(int(dg), float(rope_theta), int(wq_head_stride), int(wk_head_stride))
+    gp = seer_gate_params(int(dg), float(rope_theta), int(wq_head_stride), int(wk_head_stride), int(bool(k_maxmin)))
     _check(lib().seer_gate_scores_noalloc(ctypes.byref(sh), _ptr(q), _ptr(k), _ptr(wq), _ptr(wk), ctypes.byref(gp),
                                           _ptr(scores), _stream_ptr(stream)))
     return scores

@@ -169,7 +169,7 @@ size_t seer_workspace_bytes(int which_call, const seer_shape *shape)
     const int nb = shape->S / kBlock;
     switch (which_call) {
     case SEER_CALL_GATE_SCORES:
-        return gate_workspace_bytes(shape->B, shape->Hq, shape->Hkv, shape->S, shape->d, 256);
+        return gate_workspace_bytes(shape->B, shape->Hq, shape->Hkv, shape->S, shape->d, 256, true);
     case SEER_CALL_BLOCK_SPARSE_PREFILL:
         return 0;
     case SEER_CALL_ATTN_POOLED_MAP:
@@ -199,14 +199,21 @@ seer_status seer_gate_scores(const seer_shape *shape, const void *q, const void 
         return fail(SEER_ERR_INVALID_ARG, "q and k must be 16-byte aligned");
     if ((gp->d_gate % 4) != 0)
         return fail(SEER_ERR_UNSUPPORTED, "d_gate %d must be a multiple of 4", gp->d_gate);
-    const size_t need = gate_workspace_bytes(shape->B, shape->Hq, shape->Hkv, shape->S, shape->d, gp->d_gate);
+    if (gp->k_pooling != SEER_KPOOL_AVG && gp->k_pooling != SEER_KPOOL_MAXMIN)
+        return fail(SEER_ERR_INVALID_ARG, "unknown k_pooling %d", gp->k_pooling);
+    const bool maxmin = gp->k_pooling == SEER_KPOOL_MAXMIN;
+    if (gate_projection_smem(maxmin ? 2 * shape->d : shape->d, gp->d_gate) > 227 * 1024)
+        return fail(SEER_ERR_UNSUPPORTED, "d_gate %d too large for %s K pooling at d = %d", gp->d_gate,
+                    maxmin ? "max+min" : "average", shape->d);
+    const size_t need =
+        gate_workspace_bytes(shape->B, shape->Hq, shape->Hkv, shape->S, shape->d, gp->d_gate, maxmin);
     if (workspace == nullptr || ws_bytes < need)
         return fail(SEER_ERR_WORKSPACE, "seer_gate_scores needs %zu workspace bytes, got %zu", need, ws_bytes);
     if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
         return fail(SEER_ERR_WORKSPACE, "workspace must be 256-byte aligned");
     const cudaError_t e = launch_gate(shape->B, shape->Hq, shape->Hkv, shape->S, shape->d, gp->d_gate,
-                                      gp->rope_theta, q, k, wq, gp->wq_head_stride, wk, gp->wk_head_stride, scores,
-                                      workspace, static_cast<cudaStream_t>(stream));
+                                      gp->rope_theta, maxmin, q, k, wq, gp->wq_head_stride, wk, gp->wk_head_stride,
+                                      scores, workspace, static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess)
         return cuda_fail(e, "seer_gate_scores launch");
     return ok();

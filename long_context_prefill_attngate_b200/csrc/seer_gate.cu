@@ -24,21 +24,26 @@ namespace {
 constexpr int kPoolThreads = 128;
 
 // One CTA per (head row-group bh, block i): mean of 64 rows of d bf16 values.
-template <int D>
+// MAXMIN: per-block max and min instead of the mean, written [max | min]
+// (2D features per block) — the K pooling variant of the gate.
+template <int D, bool MAXMIN = false>
 __global__ void __launch_bounds__(kPoolThreads) pool_kernel(const __nv_bfloat16 *__restrict__ x,
                                                             float *__restrict__ out)
 {
     constexpr int CH = D / 8;                 // 16-byte chunks per row
     constexpr int RPI = kPoolThreads / CH;    // rows handled in parallel
     __shared__ float part[RPI][D];
+    __shared__ float part2[MAXMIN ? RPI : 1][MAXMIN ? D : 1];
     const long long blk = blockIdx.x;         // = bh * nb + i; the block's rows are contiguous
     const __nv_bfloat16 *base = x + blk * 64 * D;
     const int c = threadIdx.x % CH;
     const int r0 = threadIdx.x / CH;
-    float acc[8];
+    float acc[8], acc2[8];
 #pragma unroll
-    for (int e = 0; e < 8; ++e)
-        acc[e] = 0.f;
+    for (int e = 0; e < 8; ++e) {
+        acc[e] = MAXMIN ? -INFINITY : 0.f;
+        acc2[e] = INFINITY;
+    }
     uint4 vv[64 / RPI];
 #pragma unroll
     for (int it = 0; it < 64 / RPI; ++it)
@@ -49,20 +54,41 @@ __global__ void __launch_bounds__(kPoolThreads) pool_kernel(const __nv_bfloat16 
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
             const float2 f = __bfloat1622float2(h[e]);
-            acc[2 * e] += f.x;
-            acc[2 * e + 1] += f.y;
+            if (MAXMIN) {
+                acc[2 * e] = fmaxf(acc[2 * e], f.x);
+                acc[2 * e + 1] = fmaxf(acc[2 * e + 1], f.y);
+                acc2[2 * e] = fminf(acc2[2 * e], f.x);
+                acc2[2 * e + 1] = fminf(acc2[2 * e + 1], f.y);
+            } else {
+                acc[2 * e] += f.x;
+                acc[2 * e + 1] += f.y;
+            }
         }
     }
 #pragma unroll
-    for (int e = 0; e < 8; ++e)
+    for (int e = 0; e < 8; ++e) {
         part[r0][c * 8 + e] = acc[e];
+        if (MAXMIN)
+            part2[r0][c * 8 + e] = acc2[e];
+    }
     __syncthreads();
     for (int col = threadIdx.x; col < D; col += kPoolThreads) {
-        float s = 0.f;
+        if (MAXMIN) {
+            float mx = -INFINITY, mn = INFINITY;
 #pragma unroll
-        for (int r = 0; r < RPI; ++r)
-            s += part[r][col];
-        out[blk * D + col] = s * (1.0f / 64.0f);
+            for (int r = 0; r < RPI; ++r) {
+                mx = fmaxf(mx, part[r][col]);
+                mn = fminf(mn, part2[r][col]);
+            }
+            out[blk * 2 * D + col] = mx;
+            out[blk * 2 * D + D + col] = mn;
+        } else {
+            float s = 0.f;
+#pragma unroll
+            for (int r = 0; r < RPI; ++r)
+                s += part[r][col];
+            out[blk * D + col] = s * (1.0f / 64.0f);
+        }
     }
 }
 
@@ -295,49 +321,64 @@ size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 } // namespace
 
-size_t gate_workspace_bytes(int B, int Hq, int Hkv, int S, int d, int dg)
+size_t gate_workspace_bytes(int B, int Hq, int Hkv, int S, int d, int dg, bool k_maxmin)
 {
     const size_t nb = (size_t)(S / kBlock);
-    return align256(sizeof(float) * B * Hq * nb * d) + align256(sizeof(float) * B * Hkv * nb * d) +
+    const size_t dk = k_maxmin ? 2 * (size_t)d : (size_t)d;
+    return align256(sizeof(float) * B * Hq * nb * d) + align256(sizeof(float) * B * Hkv * nb * dk) +
            align256(sizeof(float) * B * Hq * nb * dg) + align256(sizeof(float) * B * Hkv * nb * dg);
 }
 
-cudaError_t launch_gate(int B, int Hq, int Hkv, int S, int d, int dg, float theta, const void *q, const void *k,
-                        const void *wq, long long wq_stride, const void *wk, long long wk_stride, float *scores,
-                        void *ws, cudaStream_t stream)
+size_t gate_projection_smem(int d_in, int dg)
+{
+    return sizeof(float) * (kProjRows * (d_in + kPStride) + (size_t)d_in * dg) + sizeof(double) * (dg / 2) + 16;
+}
+
+cudaError_t launch_gate(int B, int Hq, int Hkv, int S, int d, int dg, float theta, bool k_maxmin, const void *q,
+                        const void *k, const void *wq, long long wq_stride, const void *wk, long long wk_stride,
+                        float *scores, void *ws, cudaStream_t stream)
 {
     const int nb = S / kBlock;
+    const int dk = k_maxmin ? 2 * d : d;
     char *p = static_cast<char *>(ws);
     float *qp = reinterpret_cast<float *>(p);
     p += align256(sizeof(float) * B * Hq * (size_t)nb * d);
     float *kp = reinterpret_cast<float *>(p);
-    p += align256(sizeof(float) * B * Hkv * (size_t)nb * d);
+    p += align256(sizeof(float) * B * Hkv * (size_t)nb * dk);
     float *qt = reinterpret_cast<float *>(p);
     p += align256(sizeof(float) * B * Hq * (size_t)nb * dg);
     float *kt = reinterpret_cast<float *>(p);
 
     const auto *qb = static_cast<const __nv_bfloat16 *>(q);
     const auto *kb = static_cast<const __nv_bfloat16 *>(k);
+    const unsigned gq = (unsigned)((long long)B * Hq * nb), gk = (unsigned)((long long)B * Hkv * nb);
     if (d == 128) {
-        pool_kernel<128><<<(unsigned)((long long)B * Hq * nb), kPoolThreads, 0, stream>>>(qb, qp);
-        pool_kernel<128><<<(unsigned)((long long)B * Hkv * nb), kPoolThreads, 0, stream>>>(kb, kp);
+        pool_kernel<128><<<gq, kPoolThreads, 0, stream>>>(qb, qp);
+        if (k_maxmin)
+            pool_kernel<128, true><<<gk, kPoolThreads, 0, stream>>>(kb, kp);
+        else
+            pool_kernel<128><<<gk, kPoolThreads, 0, stream>>>(kb, kp);
     } else {
-        pool_kernel<64><<<(unsigned)((long long)B * Hq * nb), kPoolThreads, 0, stream>>>(qb, qp);
-        pool_kernel<64><<<(unsigned)((long long)B * Hkv * nb), kPoolThreads, 0, stream>>>(kb, kp);
+        pool_kernel<64><<<gq, kPoolThreads, 0, stream>>>(qb, qp);
+        if (k_maxmin)
+            pool_kernel<64, true><<<gk, kPoolThreads, 0, stream>>>(kb, kp);
+        else
+            pool_kernel<64><<<gk, kPoolThreads, 0, stream>>>(kb, kp);
     }
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess)
         return e;
-    const size_t psmem = sizeof(float) * (kProjRows * (d + kPStride) + (size_t)d * dg) + sizeof(double) * (dg / 2) + 16;
+    const size_t psmem = gate_projection_smem(dk, dg);
     e = cudaFuncSetAttribute(project_rope_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)psmem);
     if (e != cudaSuccess)
         return e;
+    const size_t psmem_q = gate_projection_smem(d, dg);
     const dim3 pg_q((nb + kProjRows - 1) / kProjRows, B * Hq);
     const dim3 pg_k((nb + kProjRows - 1) / kProjRows, B * Hkv);
-    project_rope_kernel<<<pg_q, kProjThreads, psmem, stream>>>(qp, Hq, nb, d,
+    project_rope_kernel<<<pg_q, kProjThreads, psmem_q, stream>>>(qp, Hq, nb, d,
                                                                static_cast<const __nv_bfloat16 *>(wq), wq_stride,
                                                                dg, (double)theta, qt);
-    project_rope_kernel<<<pg_k, kProjThreads, psmem, stream>>>(kp, Hkv, nb, d,
+    project_rope_kernel<<<pg_k, kProjThreads, psmem, stream>>>(kp, Hkv, nb, dk,
                                                                static_cast<const __nv_bfloat16 *>(wk), wk_stride,
                                                                dg, (double)theta, kt);
     e = cudaGetLastError();

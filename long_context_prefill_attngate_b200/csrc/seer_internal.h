@@ -34,10 +34,11 @@ cudaError_t launch_attention(const AttnLaunch &p, cudaStream_t stream);
 int attn_grid_size(int B, int Hq, int Hkv, int nb);
 
 // Gate kernels (seer_gate.cu).
-cudaError_t launch_gate(int B, int Hq, int Hkv, int S, int d, int dg, float theta, const void *q,
-                        const void *k, const void *wq, long long wq_stride, const void *wk,
-                        long long wk_stride, float *scores, void *ws, cudaStream_t stream);
-size_t gate_workspace_bytes(int B, int Hq, int Hkv, int S, int d, int dg);
+cudaError_t launch_gate(int B, int Hq, int Hkv, int S, int d, int dg, float theta, bool k_maxmin, const void *q,
+                        const void *k, const void *wq, long long wq_stride, const void *wk, long long wk_stride,
+                        float *scores, void *ws, cudaStream_t stream);
+size_t gate_workspace_bytes(int B, int Hq, int Hkv, int S, int d, int dg, bool k_maxmin);
+size_t gate_projection_smem(int d_in, int dg);
 
 // Mask / compaction kernels (seer_mask.cu).
 cudaError_t launch_mask(int B, int Hq, int nb, const float *scores, int mode, float threshold,

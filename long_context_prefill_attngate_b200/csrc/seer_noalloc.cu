@@ -10,9 +10,10 @@
 //
 // The array is a file-scope device variable of kNoAllocScratchBytes (24 MiB):
 // every GPU that loads the library holds it until the process exits.  It is
-// enough for a layer with (B*Hq + B*Hkv) * (S/64) * (d + d_gate) * 4 bytes of
-// gate workspace up to 24 MiB (for example the 32k-token Llama-3.1-8B layer,
-// 32/8 heads, d = d_gate = 128: 21 MB).  Larger shapes are rejected with
+// enough for a layer with (B*Hq*(d + d_gate) + B*Hkv*(dk + d_gate)) * (S/64) * 4
+// bytes of gate workspace up to 24 MiB, dk = d (average K pooling) or 2d
+// (max+min K pooling) — for example the 32k-token Llama-3.1-8B layer, 32/8
+// heads, d = d_gate = 128: 21 MB (23 MB with max+min).  Larger shapes are rejected with
 // SEER_ERR_UNSUPPORTED before anything is launched.
 //
 // All calls share the one array and it keeps whatever the last call left in
@@ -75,7 +76,8 @@ extern "C" seer_status seer_gate_scores_noalloc(const seer_shape *shape, const v
     // so the error text is the same; only the size limit is checked here.
     if (shape != nullptr && gp != nullptr && shape->B > 0 && shape->Hq > 0 && shape->Hkv > 0 &&
         shape->S >= kBlock && shape->d > 0 && gp->d_gate > 0) {
-        const size_t need = gate_workspace_bytes(shape->B, shape->Hq, shape->Hkv, shape->S, shape->d, gp->d_gate);
+        const size_t need = gate_workspace_bytes(shape->B, shape->Hq, shape->Hkv, shape->S, shape->d, gp->d_gate,
+                                                 gp->k_pooling == SEER_KPOOL_MAXMIN);
         if (need > kNoAllocScratchBytes)
             return set_last_error(SEER_ERR_UNSUPPORTED,
                                   "seer_gate_scores_noalloc: this shape needs %zu bytes of gate scratch; the "

@@ -207,6 +207,26 @@ def test_gate_scores(oracle, B, Hq, Hkv, S, d, dg):
     check_rel(s.cpu().numpy(), ref, "scores")
 
 
+@pytest.mark.parametrize("B,Hq,Hkv,S,d,dg", [(1, 2, 2, 512, 64, 64), (1, 8, 2, 4096, 128, 128),
+                                             (2, 5, 1, 1152, 128, 64)])
+def test_gate_scores_maxmin_k(oracle, B, Hq, Hkv, S, d, dg):
+    """K pooled by [max | min] (2d features, W_k [Hkv, 2d, dg])."""
+    w = syn.custom("gatemm", B, Hq, Hkv, S, d, number=47 + S, d_gate=dg)
+    x = syn.make_inputs(w)
+    g = torch.Generator().manual_seed(4700 + S)
+    wk = (torch.randn((Hkv, 2 * d, dg), generator=g) * (2.0 / (2 * d + dg)) ** 0.5).to(torch.bfloat16)
+    s = seer.seer_gate_scores(dev(x["q"]), dev(x["k"]), dev(x["wq"]), dev(wk), rope_theta=w.rope_theta,
+                              k_maxmin=True)
+    seer.seer_check_status()
+    ref = oracle.gate_scores(bits(x["q"]), bits(x["k"]), bits(x["wq"]), bits(wk), theta=w.rope_theta,
+                             k_maxmin=True)
+    check_rel(s.cpu().numpy(), ref, "scores(max+min K)")
+    # the same inputs through the average path must differ (the flag is honoured)
+    s_avg = seer.seer_gate_scores(dev(x["q"]), dev(x["k"]), dev(x["wq"]), dev(wk[:, :d].contiguous()),
+                                  rope_theta=w.rope_theta)
+    assert not torch.allclose(s_avg, s)
+
+
 def test_gate_scores_strong_logits(oracle):
     """Larger weights so the softmax is far from uniform (exercises exp range)."""
     w = syn.custom("gate2", 1, 4, 2, 2048, 128, number=43)

@@ -55,3 +55,18 @@ def test_gate_scores_noalloc_rejects_oversized_shape():
     st = L.seer_gate_scores_noalloc(ctypes.byref(big), fake, fake, fake, fake, ctypes.byref(gp), None, None)
     assert st == seer.SEER_ERR_UNSUPPORTED
     assert "scratch" in seer.seer_last_error()
+
+
+def test_gate_scores_noalloc_maxmin_k_matches_workspace_call():
+    """K pooled by [max | min]: the K workspace region is 2d wide."""
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    w = syn.custom("noallocmm", 1, 4, 2, 2048, 128, number=53)
+    x = syn.make_inputs(w)
+    g = torch.Generator().manual_seed(53)
+    wk = (torch.randn((2, 256, 128), generator=g) * 0.07).to(torch.bfloat16).cuda()
+    q, k, wq = (x[n].cuda().contiguous() for n in ("q", "k", "wq"))
+    a = seer.seer_gate_scores(q, k, wq, wk, rope_theta=w.rope_theta, k_maxmin=True)
+    b = seer.seer_gate_scores_noalloc(q, k, wq, wk, rope_theta=w.rope_theta, k_maxmin=True)
+    seer.seer_check_status()
+    assert torch.equal(a, b)
