@@ -85,19 +85,19 @@ def set_threads(n: int) -> None:
 
 
 def pool_avg(x: np.ndarray) -> np.ndarray:
-    """a1: mean over each 64-row block; bf16 [B,H,S,d] -> f64 [B,H,S/64,d]."""
+    """a1: mean over each 64-row block; bf16 [B,H,S,d] -> f64 [B,H,ceil(S/64),d]; the last block of a ragged S averages its real tokens."""
     x = _u16(x)
     B, H, S, d = x.shape
-    out = np.empty((B, H, S // BLOCK, d), np.float64)
+    out = np.empty((B, H, -(-S // BLOCK), d), np.float64)
     _load().oracle_pool_avg(_ptr(x), B, H, S, d, _ptr(out))
     return out
 
 
 def pool_maxmin(x: np.ndarray) -> np.ndarray:
-    """a1': per-block max and min, concatenated; bf16 [B,H,S,d] -> f64 [B,H,S/64,2d]."""
+    """a1': per-block max and min, concatenated; bf16 [B,H,S,d] -> f64 [B,H,ceil(S/64),2d]."""
     x = _u16(x)
     B, H, S, d = x.shape
-    out = np.empty((B, H, S // BLOCK, 2 * d), np.float64)
+    out = np.empty((B, H, -(-S // BLOCK), 2 * d), np.float64)
     _load().oracle_pool_maxmin(_ptr(x), B, H, S, d, _ptr(out))
     return out
 
@@ -146,7 +146,7 @@ def gate_scores(q, k, wq, wk, theta: float = 5e5, wq_head_stride=None, wk_head_s
         wq_head_stride = 0 if wq.ndim == 2 else d * dg
     if wk_head_stride is None:
         wk_head_stride = 0 if wk.ndim == 2 else dk * dg
-    nb = S // BLOCK
+    nb = -(-S // BLOCK)
     out = np.empty((B, Hq, nb, nb), np.float64)
     _load().oracle_gate_scores_kpool(_ptr(q), _ptr(k), B, Hq, Hkv, S, d, _ptr(wq), int(wq_head_stride),
                                      _ptr(wk), int(wk_head_stride), dg, float(theta), int(bool(k_maxmin)), _ptr(out))
@@ -204,12 +204,13 @@ def all_units(B: int, H: int, nb: int) -> np.ndarray:
 def masked_attention(q, k, v, mask, scale: float | None = None, units=None):
     """a6: explicit masked causal attention for the given (b,h,i) units.
 
-    Returns (o f64 [n,64,d], lse f64 [n,64]).
+    Returns (o f64 [n,64,d], lse f64 [n,64]); rows at or past S (a ragged
+    last block) are 0 with LSE -inf.
     """
     q, k, v = _u16(q), _u16(k), _u16(v)
     B, Hq, S, d = q.shape
     Hkv = k.shape[1]
-    nb = S // BLOCK
+    nb = -(-S // BLOCK)
     m = np.ascontiguousarray(mask, dtype=np.uint8)
     assert m.shape == (B, Hq, nb, nb)
     if scale is None:
@@ -228,12 +229,13 @@ def masked_attention(q, k, v, mask, scale: float | None = None, units=None):
 def pooled_map(q, k, v, scale: float | None = None, units=None):
     """a7: dense causal O plus the max-pooled map rows A[b,h,i,:].
 
-    Returns (o f64 [n,64,d], A f64 [n,nb]).
+    Returns (o f64 [n,64,d], A f64 [n,nb]); rows at or past S are 0 and do
+    not enter A.
     """
     q, k, v = _u16(q), _u16(k), _u16(v)
     B, Hq, S, d = q.shape
     Hkv = k.shape[1]
-    nb = S // BLOCK
+    nb = -(-S // BLOCK)
     if scale is None:
         scale = 1.0 / np.sqrt(d)
     if units is None:

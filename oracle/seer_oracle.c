@@ -48,6 +48,19 @@
 
 #define SEER_ORACLE_BLOCK 64 /* [SEC4]: block size fixed at 64 */
 
+/* Number of blocks of a sequence of S tokens.  When S is not a multiple of 64
+ * the last block holds the S - 64 (nb - 1) remaining tokens ([GATE Weakness
+ * 3]: the pooling is padded / ceil-mode; the reading taken is that the last
+ * block pools only its real tokens and that no query or key exists past S). */
+static int nblocks(int S) { return (S + SEER_ORACLE_BLOCK - 1) / SEER_ORACLE_BLOCK; }
+
+/* Tokens in block i of a sequence of S tokens. */
+static int block_len(int S, int i)
+{
+    const int rest = S - i * SEER_ORACLE_BLOCK;
+    return rest < SEER_ORACLE_BLOCK ? rest : SEER_ORACLE_BLOCK;
+}
+
 static double bf16_to_f64(uint16_t bits)
 {
     uint32_t u = ((uint32_t)bits) << 16;
@@ -58,12 +71,12 @@ static double bf16_to_f64(uint16_t bits)
 
 /* ---------------------------------------------------------------------------
  * a1 [GATE Weakness 3]: average pooling along the sequence axis.
- * x: bf16 [B, H, S, d]  ->  out: f64 [B, H, S/64, d]
- * out[b,h,i,c] = (1/64) * sum_{t<64} x[b,h,64 i + t, c]
+ * x: bf16 [B, H, S, d]  ->  out: f64 [B, H, nb, d], nb = ceil(S/64)
+ * out[b,h,i,c] = (1/n_i) * sum_{t<n_i} x[b,h,64 i + t, c],  n_i = tokens of block i
  * ------------------------------------------------------------------------- */
 void oracle_pool_avg(const uint16_t *x, int B, int H, int S, int d, double *out)
 {
-    const int nb = S / SEER_ORACLE_BLOCK;
+    const int nb = nblocks(S);
     const long long units = (long long)B * H * nb;
 #pragma omp parallel for schedule(static)
     for (long long u = 0; u < units; ++u) {
@@ -71,11 +84,12 @@ void oracle_pool_avg(const uint16_t *x, int B, int H, int S, int d, double *out)
         const int i = (int)(u % nb);
         const uint16_t *base = x + (bh * S + (long long)i * SEER_ORACLE_BLOCK) * d;
         double *o = out + u * d;
+        const int n = block_len(S, i);
         for (int c = 0; c < d; ++c) {
             double s = 0.0;
-            for (int t = 0; t < SEER_ORACLE_BLOCK; ++t)
+            for (int t = 0; t < n; ++t)
                 s += bf16_to_f64(base[(long long)t * d + c]);
-            o[c] = s / SEER_ORACLE_BLOCK;
+            o[c] = s / n;
         }
     }
 }
@@ -84,13 +98,13 @@ void oracle_pool_avg(const uint16_t *x, int B, int H, int S, int d, double *out)
  * a1' [GATE Weakness 3: "Max+Min pooling in K ... concated in hidden dim
  * before the linear layer ([Batch, Head, Seq / Block, Dim * 2])"; Question 1:
  * K prefers max-min pooling]:
- * out[b,h,i,c]     = max_{t<64} x[b,h,64 i + t, c]
- * out[b,h,i,d + c] = min_{t<64} x[b,h,64 i + t, c]      (max first: a reading)
- * x: bf16 [B, H, S, d]  ->  out: f64 [B, H, S/64, 2d]
+ * out[b,h,i,c]     = max_{t<n_i} x[b,h,64 i + t, c]
+ * out[b,h,i,d + c] = min_{t<n_i} x[b,h,64 i + t, c]      (max first: a reading)
+ * x: bf16 [B, H, S, d]  ->  out: f64 [B, H, nb, 2d]
  * ------------------------------------------------------------------------- */
 void oracle_pool_maxmin(const uint16_t *x, int B, int H, int S, int d, double *out)
 {
-    const int nb = S / SEER_ORACLE_BLOCK;
+    const int nb = nblocks(S);
     const long long units = (long long)B * H * nb;
 #pragma omp parallel for schedule(static)
     for (long long u = 0; u < units; ++u) {
@@ -98,9 +112,10 @@ void oracle_pool_maxmin(const uint16_t *x, int B, int H, int S, int d, double *o
         const int i = (int)(u % nb);
         const uint16_t *base = x + (bh * S + (long long)i * SEER_ORACLE_BLOCK) * d;
         double *o = out + u * 2 * d;
+        const int n = block_len(S, i);
         for (int c = 0; c < d; ++c) {
             double mx = -INFINITY, mn = INFINITY;
-            for (int t = 0; t < SEER_ORACLE_BLOCK; ++t) {
+            for (int t = 0; t < n; ++t) {
                 const double v = bf16_to_f64(base[(long long)t * d + c]);
                 if (v > mx)
                     mx = v;
@@ -204,7 +219,7 @@ void oracle_gate_scores_kpool(const uint16_t *q, const uint16_t *k, int B, int H
                               long long wk_head_stride, int dg, double theta,
                               int k_maxmin, double *scores)
 {
-    const int nb = S / SEER_ORACLE_BLOCK;
+    const int nb = nblocks(S);
     const int dk = k_maxmin ? 2 * d : d;
     double *qp = (double *)malloc(sizeof(double) * (size_t)B * Hq * nb * d);
     double *kp = (double *)malloc(sizeof(double) * (size_t)B * Hkv * nb * dk);
@@ -344,7 +359,7 @@ void oracle_masked_attention(const uint16_t *q, const uint16_t *k,
                              const int32_t *units, int n_units, double *o,
                              double *lse)
 {
-    const int nb = S / SEER_ORACLE_BLOCK;
+    const int nb = nblocks(S);
     const int g = Hq / Hkv;
     (void)B;
 #pragma omp parallel
@@ -361,6 +376,13 @@ void oracle_masked_attention(const uint16_t *q, const uint16_t *k,
             for (int t = 0; t < SEER_ORACLE_BLOCK; ++t) {
                 const int r = i * SEER_ORACLE_BLOCK + t;
                 double *orow = o + ((long long)u * SEER_ORACLE_BLOCK + t) * d;
+                if (r >= S) {
+                    /* no such query: zero row, LSE -inf */
+                    for (int e = 0; e < d; ++e)
+                        orow[e] = 0.0;
+                    lse[(long long)u * SEER_ORACLE_BLOCK + t] = -INFINITY;
+                    continue;
+                }
                 for (int c = 0; c < d; ++c)
                     qrow[c] = bf16_to_f64(qh[(long long)r * d + c]);
                 double m = -INFINITY;
@@ -413,7 +435,7 @@ void oracle_pooled_map(const uint16_t *q, const uint16_t *k, const uint16_t *v,
                        int B, int Hq, int Hkv, int S, int d, double scale,
                        const int32_t *units, int n_units, double *o, double *A)
 {
-    const int nb = S / SEER_ORACLE_BLOCK;
+    const int nb = nblocks(S);
     const int g = Hq / Hkv;
     (void)B;
 #pragma omp parallel
@@ -432,6 +454,12 @@ void oracle_pooled_map(const uint16_t *q, const uint16_t *k, const uint16_t *v,
             for (int t = 0; t < SEER_ORACLE_BLOCK; ++t) {
                 const int r = i * SEER_ORACLE_BLOCK + t;
                 double *orow = o + ((long long)u * SEER_ORACLE_BLOCK + t) * d;
+                if (r >= S) {
+                    /* no such query: zero row, no contribution to A */
+                    for (int e = 0; e < d; ++e)
+                        orow[e] = 0.0;
+                    continue;
+                }
                 for (int c = 0; c < d; ++c)
                     qrow[c] = bf16_to_f64(qh[(long long)r * d + c]);
                 double m = -INFINITY;

@@ -451,3 +451,105 @@ def test_gate_scores_maxmin_brute_force(oracle):
     # the avg path is unchanged by the new entry point
     np.testing.assert_array_equal(oracle.gate_scores(qb, kb, wqb, rand_bits((Hkv, d, dg), 96)),
                                   oracle.gate_scores(qb, kb, wqb, rand_bits((Hkv, d, dg), 96), k_maxmin=False))
+
+
+# ----------------------------------------------------- S not a multiple of 64
+def _blocks(S):
+    """(start, stop) of every 64-token block of a sequence of S tokens."""
+    return [(s, min(s + BLOCK, S)) for s in range(0, S, BLOCK)]
+
+
+def test_ragged_pool_brute_force(oracle):
+    """The last block of a ragged sequence pools only its real tokens."""
+    S = 3 * BLOCK + 17
+    bits = rand_bits((2, 3, S, 8), 101)
+    x = bits_to_f64(bits)
+    want_avg = np.stack([x[:, :, a:b].mean(2) for a, b in _blocks(S)], 2)
+    want_max = np.stack([x[:, :, a:b].max(2) for a, b in _blocks(S)], 2)
+    want_min = np.stack([x[:, :, a:b].min(2) for a, b in _blocks(S)], 2)
+    np.testing.assert_allclose(oracle.pool_avg(bits), want_avg, rtol=0, atol=1e-14)
+    mm = oracle.pool_maxmin(bits)
+    np.testing.assert_array_equal(mm[..., :8], want_max)
+    np.testing.assert_array_equal(mm[..., 8:], want_min)
+    # a constant tail block pools to that constant whatever its length
+    for tail in (1, 5, 63):
+        c = f64_to_bits(np.full((1, 1, BLOCK + tail, 4), -1.5))
+        assert np.all(oracle.pool_avg(c) == -1.5)
+
+
+def test_ragged_gate_brute_force(oracle):
+    B, Hq, Hkv, S, d, dg = 1, 4, 2, 5 * BLOCK + 9, 16, 8
+    qb, kb = rand_bits((B, Hq, S, d), 102, scale=4.0), rand_bits((B, Hkv, S, d), 103, scale=4.0, shift=0.5)
+    wqb, wkb = rand_bits((Hq, d, dg), 104, scale=0.5), rand_bits((Hkv, d, dg), 105, scale=0.5)
+    got = oracle.gate_scores(qb, kb, wqb, wkb, theta=1e3)
+    q, k = bits_to_f64(qb), bits_to_f64(kb)
+    nb = len(_blocks(S))
+    qp = np.stack([q[:, :, a:b].mean(2) for a, b in _blocks(S)], 2)
+    kp = np.stack([k[:, :, a:b].mean(2) for a, b in _blocks(S)], 2)
+    qt = np.einsum("bhid,hde->bhie", qp, bits_to_f64(wqb))
+    kt = np.einsum("bhid,hde->bhie", kp, bits_to_f64(wkb))
+    rot = np.exp(1j * np.arange(nb)[:, None] * 1e3 ** (-2.0 * np.arange(dg // 2) / dg)[None, :])
+
+    def apply(xx):
+        z = (xx[..., : dg // 2] + 1j * xx[..., dg // 2:]) * rot
+        return np.concatenate([z.real, z.imag], -1)
+
+    qt, kt = apply(qt), np.repeat(apply(kt), Hq // Hkv, axis=1)
+    lg = np.einsum("bhie,bhje->bhij", qt, kt) / math.sqrt(dg)
+    lg = np.where(np.tril(np.ones((nb, nb), bool)), lg, -np.inf)
+    e = np.exp(lg - lg.max(-1, keepdims=True))
+    assert got.shape == (B, Hq, nb, nb)
+    np.testing.assert_allclose(got, e / e.sum(-1, keepdims=True), rtol=1e-11, atol=1e-15)
+
+
+def test_ragged_attention_brute_force_and_prefix(oracle):
+    """Rows past S do not exist (zero, LSE -inf); the rest equals a token-level
+    brute force, and equals the same rows of a longer sequence (causality: a
+    token never sees later ones), whatever the extra tokens hold."""
+    B, Hq, Hkv, d = 1, 4, 2, 16
+    S = 4 * BLOCK + 21
+    nb = len(_blocks(S))
+    qb, kb, vb = (rand_bits((B, h, S, d), 106 + i, scale=1.5) for i, h in enumerate((Hq, Hkv, Hkv)))
+    m = (rng(109).random((B, Hq, nb, nb)) < 0.6).astype(np.uint8) * np.tril(np.ones((nb, nb), np.uint8))
+    m[..., np.arange(nb), np.arange(nb)] = 1
+    o, lse = oracle.masked_attention(qb, kb, vb, m, scale=0.2)
+    q, k, v = bits_to_f64(qb), bits_to_f64(kb), bits_to_f64(vb)
+    blk = np.arange(S) // BLOCK
+    o = o.reshape(B, Hq, nb * BLOCK, d)
+    lse = lse.reshape(B, Hq, nb * BLOCK)
+    for h in range(Hq):
+        tok = m[0, h][blk[:, None], blk[None, :]].astype(bool) & np.tril(np.ones((S, S), bool))
+        s = np.where(tok, q[0, h] @ k[0, h // 2].T * 0.2, -np.inf)
+        mx = s.max(-1, keepdims=True)
+        p = np.exp(s - mx)
+        np.testing.assert_allclose(o[0, h, :S], (p @ v[0, h // 2]) / p.sum(-1, keepdims=True), rtol=1e-10,
+                                   atol=1e-12)
+        np.testing.assert_allclose(lse[0, h, :S], (mx + np.log(p.sum(-1, keepdims=True)))[:, 0], rtol=1e-12)
+    assert np.all(o[:, :, S:] == 0) and np.all(np.isneginf(lse[:, :, S:]))
+    # the same rows of a block-aligned sequence with arbitrary extra tokens
+    pad = nb * BLOCK - S
+    ext = [np.concatenate([t, rand_bits((B, t.shape[1], pad, d), 110 + i, scale=9.0)], 2)
+           for i, t in enumerate((qb, kb, vb))]
+    o2, lse2 = oracle.masked_attention(*ext, m, scale=0.2)
+    np.testing.assert_array_equal(o2.reshape(B, Hq, nb * BLOCK, d)[:, :, :S], o[:, :, :S])
+    np.testing.assert_array_equal(lse2.reshape(B, Hq, nb * BLOCK)[:, :, :S], lse[:, :, :S])
+
+
+def test_ragged_pooled_map_brute_force(oracle):
+    B, Hq, Hkv, d = 1, 2, 1, 16
+    S = 4 * BLOCK + 30
+    nb = len(_blocks(S))
+    qb, kb, vb = (rand_bits((B, h, S, d), 112 + i, scale=2.0) for i, h in enumerate((Hq, Hkv, Hkv)))
+    o, A = oracle.pooled_map(qb, kb, vb)
+    q, k, v = bits_to_f64(qb), bits_to_f64(kb), bits_to_f64(vb)
+    A = A.reshape(Hq, nb, nb)
+    o = o.reshape(Hq, nb * BLOCK, d)
+    for h in range(Hq):
+        s = q[0, h] @ k[0, 0].T / 4.0 + np.triu(np.full((S, S), -np.inf), 1)
+        p = np.exp(s - s.max(-1, keepdims=True))
+        p /= p.sum(-1, keepdims=True)
+        np.testing.assert_allclose(o[h, :S], p @ v[0, 0], rtol=1e-10, atol=1e-12)
+        assert np.all(o[h, S:] == 0)
+        want = np.array([[p[a:b, c:e].max() if j <= i else 0.0 for j, (c, e) in enumerate(_blocks(S))]
+                         for i, (a, b) in enumerate(_blocks(S))])
+        np.testing.assert_allclose(A[h], want, rtol=1e-12, atol=0)
