@@ -30,8 +30,12 @@
  *    ran out) are recorded in a device status word and reported by
  *    seer_check_status().
  *  - seer_last_error() returns a thread-local text for the last failure.
- *  - Supported: S % 64 == 0 (S >= 64), S/64 <= 16384, d in {64, 128},
+ *  - Supported: any S >= 1 with nb = ceil(S/64) <= 16384, d in {64, 128},
  *    Hq % Hkv == 0.  Other shapes return SEER_ERR_UNSUPPORTED.
+ *  - S not a multiple of 64 ("Learning Intrinsic Sparse Attention",
+ *    rebuttal Weakness 3: padded, ceil-mode pooling): the last block holds
+ *    the S - 64 (nb - 1) remaining tokens; it pools only those tokens, and no
+ *    query or key exists past S (rows past S are never written).
  */
 #ifndef SEER_H
 #define SEER_H
@@ -59,7 +63,7 @@ typedef enum seer_status {
     SEER_ERR_DEVICE = 6        /* another device-side check failed          */
 } seer_status;
 
-/* Problem shape.  nb = S / 64 query/key blocks. */
+/* Problem shape.  nb = ceil(S / 64) query/key blocks. */
 typedef struct seer_shape {
     int B, Hq, Hkv, S, d;
 } seer_shape;
@@ -113,7 +117,7 @@ enum {
  * the sequence axis, [B, H, S/64, d], before the linear layer; Q1: block
  * RoPE on the non-RoPE'd pooled Q/K; Weakness 2: softmax like attention
  * without V; Question 2: rows sum to 1.)
- *   Qp = mean over each 64-token block of q   (K likewise: average pooling)
+ *   Qp = mean over each block's tokens of q   (K likewise: average pooling)
  *   Qt = RoPE_i(Qp @ Wq[h]),  Kt = RoPE_j(Kp @ Wk[h_kv])
  *   scores[b,h,i,j] = softmax_{j<=i}(Qt_i . Kt_j / sqrt(d_gate)); 0 for j > i.
  * With k_pooling = SEER_KPOOL_MAXMIN, Kp = [max | min] over each block (2d

@@ -173,7 +173,7 @@ def seer_gate_scores(q, k, wq, wk, rope_theta: float = 5e5, scores=None, workspa
     _need(q.dtype == k.dtype == wq.dtype == wk.dtype == torch.bfloat16, "q, k, wq, wk must be bf16")
     sh = shape_of(q, k)
     d, dg = sh.d, wq.shape[-1]
-    nb = sh.S // BLOCK
+    nb = -(-sh.S // BLOCK)
     if wq_head_stride is None:
         wq_head_stride = 0 if wq.dim() == 2 else d * dg
     if wk_head_stride is None:
@@ -200,7 +200,7 @@ def seer_gate_scores_noalloc(q, k, wq, wk, rope_theta: float = 5e5, scores=None,
           "tensors must be contiguous")
     sh = shape_of(q, k)
     d, dg = sh.d, wq.shape[-1]
-    nb = sh.S // BLOCK
+    nb = -(-sh.S // BLOCK)
     if wq_head_stride is None:
         wq_head_stride = 0 if wq.dim() == 2 else d * dg
     if wk_head_stride is None:
@@ -273,7 +273,7 @@ def seer_attn_pooled_map(q, k, v, softmax_scale: float = 0.0, o=None, A=None, wo
     _need(all(t.is_contiguous() for t in (q, k, v)), "tensors must be contiguous")
     _need(q.dtype == k.dtype == v.dtype == torch.bfloat16, "bf16 q/k/v")
     sh = shape_of(q, k)
-    nb = sh.S // BLOCK
+    nb = -(-sh.S // BLOCK)
     if o is None:
         o = torch.empty_like(q)
     if A is None:

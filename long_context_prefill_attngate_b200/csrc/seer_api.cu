@@ -55,12 +55,10 @@ seer_status check_shape(const seer_shape *sh)
                     sh->Hq, sh->Hkv, sh->S, sh->d);
     if (sh->Hq % sh->Hkv != 0)
         return fail(SEER_ERR_INVALID_ARG, "Hq (%d) must be a multiple of Hkv (%d)", sh->Hq, sh->Hkv);
-    if (sh->S % kBlock != 0)
-        return fail(SEER_ERR_UNSUPPORTED, "S (%d) must be a multiple of 64", sh->S);
     if (sh->d != 64 && sh->d != 128)
         return fail(SEER_ERR_UNSUPPORTED, "head dim %d not supported (64 or 128)", sh->d);
-    if (sh->S / kBlock > kMaxNb)
-        return fail(SEER_ERR_UNSUPPORTED, "S/64 = %d exceeds %d", sh->S / kBlock, kMaxNb);
+    if (num_blocks(sh->S) > kMaxNb)
+        return fail(SEER_ERR_UNSUPPORTED, "ceil(S/64) = %d exceeds %d", num_blocks(sh->S), kMaxNb);
     if ((long long)sh->B * sh->Hq > (1LL << 30) / kMaxNb)
         return fail(SEER_ERR_UNSUPPORTED, "B*Hq too large");
     return SEER_OK;
@@ -166,7 +164,7 @@ size_t seer_workspace_bytes(int which_call, const seer_shape *shape)
 {
     if (check_shape(shape) != SEER_OK)
         return 0;
-    const int nb = shape->S / kBlock;
+    const int nb = num_blocks(shape->S);
     switch (which_call) {
     case SEER_CALL_GATE_SCORES:
         return gate_workspace_bytes(shape->B, shape->Hq, shape->Hkv, shape->S, shape->d, 256, true);
@@ -234,7 +232,7 @@ seer_status seer_block_mask(const seer_shape *shape, const float *scores, const 
         return fail(SEER_ERR_INVALID_ARG, "TopK density must be finite and >= 0");
     if (mp->mode == SEER_MASK_THRESHOLD && std::isnan(mp->threshold))
         return fail(SEER_ERR_INVALID_ARG, "threshold is NaN");
-    const cudaError_t e = launch_mask(shape->B, shape->Hq, shape->S / kBlock, scores, mp->mode, mp->threshold,
+    const cudaError_t e = launch_mask(shape->B, shape->Hq, num_blocks(shape->S), scores, mp->mode, mp->threshold,
                                       mp->density, mp->k_fixed, mp->k_per_row, mp->force_first ? 1 : 0,
                                       mp->force_diag ? 1 : 0, mask, static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess)
@@ -251,7 +249,7 @@ seer_status seer_compact_mask(const seer_shape *shape, const uint8_t *mask, int3
     if (mask == nullptr || lists == nullptr || counts == nullptr)
         return fail(SEER_ERR_INVALID_ARG, "seer_compact_mask: NULL argument");
     const cudaError_t e =
-        launch_compact(shape->B, shape->Hq, shape->S / kBlock, mask, lists, counts, static_cast<cudaStream_t>(stream));
+        launch_compact(shape->B, shape->Hq, num_blocks(shape->S), mask, lists, counts, static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess)
         return cuda_fail(e, "seer_compact_mask launch");
     return ok();
@@ -292,7 +290,7 @@ seer_status seer_block_sparse_prefill(const seer_shape *shape, const void *q, co
     a.Hkv = shape->Hkv;
     a.S = shape->S;
     a.d = shape->d;
-    a.nb = shape->S / kBlock;
+    a.nb = num_blocks(shape->S);
     const float scale = softmax_scale > 0.f ? softmax_scale : 1.0f / sqrtf((float)shape->d);
     a.scale_log2 = scale * 1.4426950408889634f;
     a.mask = mask;
@@ -321,7 +319,7 @@ seer_status seer_attn_pooled_map(const seer_shape *shape, const void *q, const v
         return fail(SEER_ERR_INVALID_ARG, "seer_attn_pooled_map: NULL A");
     if (std::isnan(softmax_scale) || std::isinf(softmax_scale))
         return fail(SEER_ERR_INVALID_ARG, "softmax_scale must be finite");
-    const int nb = shape->S / kBlock;
+    const int nb = num_blocks(shape->S);
     const int grid = attn_grid_size(shape->B, shape->Hq, shape->Hkv, nb);
     const size_t need = sizeof(float) * (size_t)grid * nb * 128;
     if (workspace == nullptr || ws_bytes < need)
@@ -365,7 +363,7 @@ seer_status seer_distill_loss(const seer_shape *shape, const float *scores, cons
         return st;
     if (scores == nullptr || A == nullptr || loss_rows == nullptr || loss == nullptr)
         return fail(SEER_ERR_INVALID_ARG, "seer_distill_loss: NULL scores, A, loss_rows or loss");
-    const cudaError_t e = launch_distill(shape->B, shape->Hq, shape->S / kBlock, scores, A, A_norm, loss_rows, loss,
+    const cudaError_t e = launch_distill(shape->B, shape->Hq, num_blocks(shape->S), scores, A, A_norm, loss_rows, loss,
                                          static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess)
         return cuda_fail(e, "seer_distill_loss launch");

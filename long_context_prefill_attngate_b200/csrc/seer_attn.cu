@@ -620,6 +620,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                 }
                 tc_fence_after();
             }
+            // A ragged last block has rows past S: they were computed from the
+            // zero rows TMA fills in, and are neither stored nor pooled (the
+            // TMEM reads below stay warp-uniform; only the stores are per row).
+            const bool row_ok = present && my_i * 64 + r_in < p.S;
             if (present) {
                 const size_t orow = ((size_t)(inf.b * p.Hq + my_h) * p.S + (size_t)my_i * 64 + r_in);
                 uint4 *dst = reinterpret_cast<uint4 *>(p.o + orow * D);
@@ -639,11 +643,14 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                         const float a1 = has ? __uint_as_float(ov[2 * c + 1]) * inv_l : 0.f;
                         pkd[c] = pack_bf16x2(a0, a1);
                     }
+                    if (row_ok) {
 #pragma unroll
-                    for (int v4 = 0; v4 < 4; ++v4)
-                        dst[ch * 4 + v4] = make_uint4(pkd[4 * v4], pkd[4 * v4 + 1], pkd[4 * v4 + 2], pkd[4 * v4 + 3]);
+                        for (int v4 = 0; v4 < 4; ++v4)
+                            dst[ch * 4 + v4] =
+                                make_uint4(pkd[4 * v4], pkd[4 * v4 + 1], pkd[4 * v4 + 2], pkd[4 * v4 + 3]);
+                    }
                 }
-                if (p.lse != nullptr)
+                if (p.lse != nullptr && row_ok)
                     p.lse[orow] = has ? (m + __log2f(l)) * 0.69314718055994530942f : -INFINITY;
             }
             if (inf.count > 0) {
@@ -652,14 +659,14 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             }
             if (MAP) {
                 // Figure 8 second pass: a_ij = 2^(r_ij - m) / l, A_ij = max over the 64 rows.
-                const float inv_l = (present && l > 0.f) ? 1.0f / l : 0.f;
+                const float inv_l = (row_ok && l > 0.f) ? 1.0f / l : 0.f;
                 float *Arow = present ? p.A + ((size_t)(inf.b * p.Hq + my_h) * p.nb + my_i) * p.nb : nullptr;
                 for (int t0 = 0; t0 < inf.count; t0 += 32) {
                     float vals[32];
 #pragma unroll
                     for (int k = 0; k < 32; ++k) {
                         const int t = t0 + k;
-                        vals[k] = (present && t < inf.count && t <= my_i)
+                        vals[k] = (row_ok && t < inf.count && t <= my_i)
                                       ? ex2_approx(rs[(size_t)t * kRows + row] - m) * inv_l
                                       : 0.f;
                     }

@@ -23,19 +23,23 @@ namespace {
 
 constexpr int kPoolThreads = 128;
 
-// One CTA per (head row-group bh, block i): mean of 64 rows of d bf16 values.
+// One CTA per (head row-group bh, block i): mean of the block's rows of d
+// bf16 values (64, or the S - 64 i tokens of a ragged last block).
 // MAXMIN: per-block max and min instead of the mean, written [max | min]
 // (2D features per block) — the K pooling variant of the gate.
 template <int D, bool MAXMIN = false>
-__global__ void __launch_bounds__(kPoolThreads) pool_kernel(const __nv_bfloat16 *__restrict__ x,
+__global__ void __launch_bounds__(kPoolThreads) pool_kernel(const __nv_bfloat16 *__restrict__ x, int S, int nb,
                                                             float *__restrict__ out)
 {
     constexpr int CH = D / 8;                 // 16-byte chunks per row
     constexpr int RPI = kPoolThreads / CH;    // rows handled in parallel
     __shared__ float part[RPI][D];
     __shared__ float part2[MAXMIN ? RPI : 1][MAXMIN ? D : 1];
-    const long long blk = blockIdx.x;         // = bh * nb + i; the block's rows are contiguous
-    const __nv_bfloat16 *base = x + blk * 64 * D;
+    const long long blk = blockIdx.x;         // = bh * nb + i
+    const long long bh = blk / nb;
+    const int i = (int)(blk % nb);
+    const int rows = min(64, S - 64 * i);      // tokens in this block
+    const __nv_bfloat16 *base = x + (bh * S + 64LL * i) * D;
     const int c = threadIdx.x % CH;
     const int r0 = threadIdx.x / CH;
     float acc[8], acc2[8];
@@ -47,9 +51,12 @@ __global__ void __launch_bounds__(kPoolThreads) pool_kernel(const __nv_bfloat16 
     uint4 vv[64 / RPI];
 #pragma unroll
     for (int it = 0; it < 64 / RPI; ++it)
-        vv[it] = __ldg(reinterpret_cast<const uint4 *>(base + (size_t)(r0 + it * RPI) * D) + c);
+        if (rows == 64 || r0 + it * RPI < rows)
+            vv[it] = __ldg(reinterpret_cast<const uint4 *>(base + (size_t)(r0 + it * RPI) * D) + c);
 #pragma unroll
     for (int it = 0; it < 64 / RPI; ++it) {
+        if (rows != 64 && r0 + it * RPI >= rows)
+            continue;
         const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&vv[it]);
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
@@ -87,7 +94,7 @@ __global__ void __launch_bounds__(kPoolThreads) pool_kernel(const __nv_bfloat16 
 #pragma unroll
             for (int r = 0; r < RPI; ++r)
                 s += part[r][col];
-            out[blk * D + col] = s * (1.0f / 64.0f);
+            out[blk * D + col] = s / (float)rows;
         }
     }
 }
@@ -323,7 +330,7 @@ size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 size_t gate_workspace_bytes(int B, int Hq, int Hkv, int S, int d, int dg, bool k_maxmin)
 {
-    const size_t nb = (size_t)(S / kBlock);
+    const size_t nb = (size_t)num_blocks(S);
     const size_t dk = k_maxmin ? 2 * (size_t)d : (size_t)d;
     return align256(sizeof(float) * B * Hq * nb * d) + align256(sizeof(float) * B * Hkv * nb * dk) +
            align256(sizeof(float) * B * Hq * nb * dg) + align256(sizeof(float) * B * Hkv * nb * dg);
@@ -338,7 +345,7 @@ cudaError_t launch_gate(int B, int Hq, int Hkv, int S, int d, int dg, float thet
                         const void *k, const void *wq, long long wq_stride, const void *wk, long long wk_stride,
                         float *scores, void *ws, cudaStream_t stream)
 {
-    const int nb = S / kBlock;
+    const int nb = num_blocks(S);
     const int dk = k_maxmin ? 2 * d : d;
     char *p = static_cast<char *>(ws);
     float *qp = reinterpret_cast<float *>(p);
@@ -353,17 +360,17 @@ cudaError_t launch_gate(int B, int Hq, int Hkv, int S, int d, int dg, float thet
     const auto *kb = static_cast<const __nv_bfloat16 *>(k);
     const unsigned gq = (unsigned)((long long)B * Hq * nb), gk = (unsigned)((long long)B * Hkv * nb);
     if (d == 128) {
-        pool_kernel<128><<<gq, kPoolThreads, 0, stream>>>(qb, qp);
+        pool_kernel<128><<<gq, kPoolThreads, 0, stream>>>(qb, S, nb, qp);
         if (k_maxmin)
-            pool_kernel<128, true><<<gk, kPoolThreads, 0, stream>>>(kb, kp);
+            pool_kernel<128, true><<<gk, kPoolThreads, 0, stream>>>(kb, S, nb, kp);
         else
-            pool_kernel<128><<<gk, kPoolThreads, 0, stream>>>(kb, kp);
+            pool_kernel<128><<<gk, kPoolThreads, 0, stream>>>(kb, S, nb, kp);
     } else {
-        pool_kernel<64><<<gq, kPoolThreads, 0, stream>>>(qb, qp);
+        pool_kernel<64><<<gq, kPoolThreads, 0, stream>>>(qb, S, nb, qp);
         if (k_maxmin)
-            pool_kernel<64, true><<<gk, kPoolThreads, 0, stream>>>(kb, kp);
+            pool_kernel<64, true><<<gk, kPoolThreads, 0, stream>>>(kb, S, nb, kp);
         else
-            pool_kernel<64><<<gk, kPoolThreads, 0, stream>>>(kb, kp);
+            pool_kernel<64><<<gk, kPoolThreads, 0, stream>>>(kb, S, nb, kp);
     }
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess)

@@ -11,6 +11,10 @@
 namespace seer {
 
 constexpr int kBlock = 64;            // block size of gate, mask and kernels
+
+// Blocks of a sequence of S tokens; the last one holds S - 64 (nb - 1) tokens
+// when S is not a multiple of 64.
+inline int num_blocks(int S) { return (S + kBlock - 1) / kBlock; }
 constexpr int kMaxNb = 16384;         // S <= 1M tokens
 constexpr int kMaxAttnCtas = 296;     // tile pipelines in flight: 2 slots x 148 SMs
 constexpr int kAttnThreads = 512;     // 2 slots x (4 softmax + Q/K producer + MMA + list builder + V producer) warps

@@ -75,7 +75,7 @@ extern "C" seer_status seer_gate_scores_noalloc(const seer_shape *shape, const v
     // Shapes the workspace call would reject are passed on to it unchanged,
     // so the error text is the same; only the size limit is checked here.
     if (shape != nullptr && gp != nullptr && shape->B > 0 && shape->Hq > 0 && shape->Hkv > 0 &&
-        shape->S >= kBlock && shape->d > 0 && gp->d_gate > 0) {
+        shape->S > 0 && shape->d > 0 && gp->d_gate > 0) {
         const size_t need = gate_workspace_bytes(shape->B, shape->Hq, shape->Hkv, shape->S, shape->d, gp->d_gate,
                                                  gp->k_pooling == SEER_KPOOL_MAXMIN);
         if (need > kNoAllocScratchBytes)

@@ -53,7 +53,7 @@ class Workload:
 
     @property
     def nb(self) -> int:
-        return self.S // BLOCK
+        return -(-self.S // BLOCK)      # the last block is partial when S % 64 != 0
 
     @property
     def seed(self) -> int:
@@ -100,7 +100,7 @@ def make_inputs(w: Workload, seed: int | None = None) -> dict:
     v = torch.randn((w.B, w.Hkv, w.S, w.d), generator=g, dtype=torch.float32)
     if w.block_bias:
         bias = torch.randn((w.B, w.Hkv, w.nb, 1, w.d), generator=g, dtype=torch.float32) * 0.5
-        k = (k.view(w.B, w.Hkv, w.nb, BLOCK, w.d) + bias).view(w.B, w.Hkv, w.S, w.d)
+        k = k + bias[:, :, :, 0].repeat_interleave(BLOCK, dim=2)[:, :, : w.S]
         k[:, :, :BLOCK, :] *= 3.0
     bound = math.sqrt(6.0 / (w.d + w.d_gate))
     wq = (torch.rand((w.Hq, w.d, w.d_gate), generator=g, dtype=torch.float32) * 2 - 1) * bound

@@ -51,7 +51,7 @@ def test_workspace_sizes(L):
 
 
 @pytest.mark.parametrize("shape,status,msg", [
-    ((1, 32, 8, 100, 128), seer.SEER_ERR_UNSUPPORTED, "multiple of 64"),
+    ((1, 2, 2, 64 * 16384 + 1, 64), seer.SEER_ERR_UNSUPPORTED, "exceeds"),
     ((1, 32, 8, 4096, 96), seer.SEER_ERR_UNSUPPORTED, "head dim"),
     ((1, 30, 8, 4096, 128), seer.SEER_ERR_INVALID_ARG, "multiple of Hkv"),
     ((0, 32, 8, 4096, 128), seer.SEER_ERR_INVALID_ARG, "positive"),
@@ -105,3 +105,12 @@ def test_topk_counts_helper_matches_oracle(oracle):
         got = seer.topk_counts(density, 300)
         want = oracle.topk_counts(density, 300)
         assert list(got) == list(want)
+
+
+def test_ragged_sequence_accepted(L):
+    """S that is not a multiple of 64: nb = ceil(S/64), the gate workspace
+    covers that many blocks and the shape passes the argument checks."""
+    sh = seer.seer_shape(1, 4, 2, 100, 64)
+    ws = seer.seer_workspace_bytes(seer.SEER_CALL_GATE_SCORES, sh)
+    assert ws >= 4 * (4 * 2 * (64 + 256) + 2 * 2 * (128 + 256))
+    assert seer.seer_workspace_bytes(seer.SEER_CALL_ATTN_POOLED_MAP, sh) == 4 * 296 * 2 * 128

@@ -66,9 +66,17 @@ def units_all(B, H, nb):
     return oracle.all_units(B, H, nb)
 
 
-def gather_units(t, units):
-    """Rows [n, 64, ...] of a [B,H,S,...] tensor for (b, h, i) units."""
-    return torch.stack([t[b, h, i * BLOCK:(i + 1) * BLOCK] for b, h, i in units])
+def gather_units(t, units, fill=0.0):
+    """Rows [n, 64, ...] of a [B,H,S,...] tensor for (b, h, i) units; the rows
+    a ragged last block lacks (past S) are filled with `fill`, as the oracle
+    reports them."""
+    out = []
+    for b, h, i in units:
+        r = t[b, h, i * BLOCK:(i + 1) * BLOCK]
+        if r.shape[0] < BLOCK:
+            r = torch.cat([r, torch.full((BLOCK - r.shape[0],) + tuple(r.shape[1:]), fill, dtype=r.dtype)])
+        out.append(r)
+    return torch.stack(out)
 
 
 def sample_units(B, H, nb, n_blocks, seed):
@@ -83,12 +91,12 @@ def run_prefill_case(oracle, q, k, v, mask, units=None, scale=0.0, lse=True):
     seer.seer_check_status()
     B, Hq, S, d = q.shape
     if units is None:
-        units = units_all(B, Hq, S // BLOCK)
+        units = units_all(B, Hq, -(-S // BLOCK))
     o_ref, lse_ref = oracle.masked_attention(bits(q), bits(k), bits(v), mask.numpy(),
                                              scale=(scale if scale > 0 else None), units=units)
     check_o(gather_units(o.cpu(), units), o_ref, "O")
     if lse:
-        lg = gather_units(l.cpu(), units).double().numpy()
+        lg = gather_units(l.cpu(), units, fill=float("-inf")).double().numpy()
         fin = np.isfinite(lse_ref)
         assert np.array_equal(np.isfinite(lg), fin)
         assert np.abs(lg[fin] - lse_ref[fin]).max() <= 1e-3
@@ -116,6 +124,63 @@ def test_prefill_shapes(oracle, B, Hq, Hkv, S, d, p, ff, fd):
     x = syn.make_inputs(w)
     mask = syn.random_mask(B, Hq, S // BLOCK, p, seed=S + Hq, force_first=ff, force_diag=fd)
     run_prefill_case(oracle, x["q"], x["k"], x["v"], mask)
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,S,d,p", [
+    (1, 4, 2, 5 * BLOCK + 17, 128, 0.5),      # ragged last block, head pairs
+    (2, 3, 1, 3 * BLOCK + 1, 64, 0.6),        # a one-token last block, leftover head
+    (1, 8, 2, 9 * BLOCK + 63, 128, 0.3),      # 63 of 64
+    (1, 2, 2, 37, 64, 1.0),                   # S < 64: one partial block
+    (1, 6, 2, 20 * BLOCK + 40, 128, 1.0),     # dense causal, ragged
+])
+def test_prefill_ragged_sequence(oracle, B, Hq, Hkv, S, d, p):
+    """S not a multiple of 64: rows past S are never written, keys past S never
+    attended (TMA fills them with zeros; the causal mask of the last block
+    excludes them)."""
+    w = syn.custom("ragged", B, Hq, Hkv, S, d, number=211 + S)
+    x = syn.make_inputs(w)
+    nb = -(-S // BLOCK)
+    mask = syn.random_mask(B, Hq, nb, p, seed=S + 5)
+    qd, kd, vd = dev(x["q"]), dev(x["k"]), dev(x["v"])
+    # O as a view at the front of a larger buffer: rows a kernel wrote past S
+    # of the last head would land in the sentinel tail.
+    n = B * Hq * S * d
+    flat = torch.full((n + BLOCK * d,), 7.0, dtype=torch.bfloat16, device="cuda")
+    seer.seer_block_sparse_prefill(qd, kd, vd, dev(mask), o=flat[:n].view(B, Hq, S, d))
+    seer.seer_check_status()
+    assert torch.all(flat[n:] == 7.0)
+    run_prefill_case(oracle, x["q"], x["k"], x["v"], mask)
+
+
+def test_pooled_map_ragged_sequence(oracle):
+    B, Hq, Hkv, S, d = 1, 4, 2, 7 * BLOCK + 29, 128
+    w = syn.custom("rmap", B, Hq, Hkv, S, d, number=223)
+    x = syn.make_inputs(w)
+    o, A = seer.seer_attn_pooled_map(dev(x["q"]), dev(x["k"]), dev(x["v"]))
+    seer.seer_check_status()
+    nb = -(-S // BLOCK)
+    units = units_all(B, Hq, nb)
+    o_ref, A_ref = oracle.pooled_map(bits(x["q"]), bits(x["k"]), bits(x["v"]), units=units)
+    check_o(gather_units(o.cpu(), units), o_ref, "O(map, ragged)")
+    check_rel(A.cpu().numpy().reshape(-1, nb), A_ref, "A(ragged)")
+
+
+@pytest.mark.parametrize("S,maxmin", [(4 * BLOCK + 3, False), (9 * BLOCK + 50, True), (50, False)])
+def test_gate_scores_ragged_sequence(oracle, S, maxmin):
+    B, Hq, Hkv, d, dg = 1, 4, 2, 128, 64
+    w = syn.custom("rgate", B, Hq, Hkv, S, d, number=227 + S, d_gate=dg)
+    x = syn.make_inputs(w)
+    wk = x["wk"]
+    if maxmin:
+        g = torch.Generator().manual_seed(S)
+        wk = (torch.randn((Hkv, 2 * d, dg), generator=g) * 0.08).to(torch.bfloat16)
+    s = seer.seer_gate_scores(dev(x["q"]), dev(x["k"]), dev(x["wq"]), dev(wk), rope_theta=w.rope_theta,
+                              k_maxmin=maxmin)
+    seer.seer_check_status()
+    ref = oracle.gate_scores(bits(x["q"]), bits(x["k"]), bits(x["wq"]), bits(wk), theta=w.rope_theta,
+                             k_maxmin=maxmin)
+    assert s.shape[-1] == -(-S // BLOCK)
+    check_rel(s.cpu().numpy(), ref, "scores(ragged)")
 
 
 def test_prefill_all_zero_mask_gives_zero_output(oracle):
