@@ -188,13 +188,14 @@ __global__ void __launch_bounds__(kProjThreads)
     }
 }
 
-constexpr int kLR = 64;              // query blocks per CTA
+constexpr int kLR = 32;              // query blocks per CTA
+constexpr int kLA = kLR / 16;        // query rows per thread
 constexpr int kLC = 64;              // key blocks per tile
 constexpr int kLThreads = 256;       // 16 x 16: rows ty + 16a, columns tx + 16b
 constexpr int kLPad = 4;             // row padding (floats): conflict-free float4 reads
 
-// Causal block logits + row softmax for 64 query blocks of one head.  Each
-// thread computes 4 x 4 logits per 64 x 64 tile from float4 reads of the
+// Causal block logits + row softmax for kLR query blocks of one head.  Each
+// thread computes kLA x 4 logits per kLR x 64 tile from float4 reads of the
 // shared Qt and Kt rows; raw logits (times 1/sqrt(dg)) go to `scores` while
 // each row's running max and exp-sum are kept online (the 16 threads sharing
 // a row reduce with shuffles).  A second pass over the same tiles writes
@@ -207,10 +208,11 @@ __global__ void __launch_bounds__(kLThreads)
     const int rs = dg + kLPad;
     float *sq = reinterpret_cast<float *>(gsm4);           // kLR x rs
     float *sk = sq + kLR * rs;                             // kLC x rs
-    const int bh = blockIdx.y;                             // b * Hq + h
+    const int bh = blockIdx.x;                             // b * Hq + h
     const int b = bh / Hq, h = bh % Hq;
     const int g = Hq / Hkv;
-    const int i0 = blockIdx.x * kLR;
+    // Heaviest query chunks (most causal columns) of every head first.
+    const int i0 = (gridDim.y - 1 - blockIdx.y) * kLR;
     const int rows = min(kLR, nb - i0);
     const float *qbase = qt + ((long long)bh * nb + i0) * dg;
     const float *kbase = kt + ((long long)(b * Hkv + h / g) * nb) * dg;
@@ -223,9 +225,9 @@ __global__ void __launch_bounds__(kLThreads)
     }
     const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
     const int jlast = i0 + rows - 1;
-    float m[4], ssum[4];
+    float m[kLA], ssum[kLA];
 #pragma unroll
-    for (int a = 0; a < 4; ++a) {
+    for (int a = 0; a < kLA; ++a) {
         m[a] = -INFINITY;
         ssum[a] = 0.f;
     }
@@ -239,30 +241,30 @@ __global__ void __launch_bounds__(kLThreads)
             *reinterpret_cast<float4 *>(sk + jj * rs + 4 * c4) = v;
         }
         __syncthreads();
-        float acc[4][4];
+        float acc[kLA][4];
 #pragma unroll
-        for (int a = 0; a < 4; ++a)
+        for (int a = 0; a < kLA; ++a)
 #pragma unroll
             for (int c = 0; c < 4; ++c)
                 acc[a][c] = 0.f;
 #pragma unroll 2
         for (int c = 0; c < dg; c += 4) {
-            float4 qv[4], kv[4];
+            float4 qv[kLA], kv[4];
 #pragma unroll
-            for (int a = 0; a < 4; ++a)
+            for (int a = 0; a < kLA; ++a)
                 qv[a] = *reinterpret_cast<const float4 *>(sq + (ty + 16 * a) * rs + c);
 #pragma unroll
             for (int bb = 0; bb < 4; ++bb)
                 kv[bb] = *reinterpret_cast<const float4 *>(sk + (tx + 16 * bb) * rs + c);
 #pragma unroll
-            for (int a = 0; a < 4; ++a)
+            for (int a = 0; a < kLA; ++a)
 #pragma unroll
                 for (int bb = 0; bb < 4; ++bb)
                     acc[a][bb] = fmaf(qv[a].x, kv[bb].x,
                                       fmaf(qv[a].y, kv[bb].y, fmaf(qv[a].z, kv[bb].z, fmaf(qv[a].w, kv[bb].w, acc[a][bb]))));
         }
 #pragma unroll
-        for (int a = 0; a < 4; ++a) {
+        for (int a = 0; a < kLA; ++a) {
             const int r = ty + 16 * a;
             const int i = i0 + r;
             float tm = -INFINITY;
@@ -298,7 +300,7 @@ __global__ void __launch_bounds__(kLThreads)
     // Normalise: each thread rereads exactly the logits it wrote.
     for (int j0 = 0; j0 <= jlast; j0 += kLC) {
 #pragma unroll
-        for (int a = 0; a < 4; ++a) {
+        for (int a = 0; a < kLA; ++a) {
             const int r = ty + 16 * a;
             const int i = i0 + r;
             if (r >= rows)
@@ -395,7 +397,7 @@ cudaError_t launch_gate(int B, int Hq, int Hkv, int S, int d, int dg, float thet
     e = cudaFuncSetAttribute(gate_softmax_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ssmem);
     if (e != cudaSuccess)
         return e;
-    const dim3 sg((nb + kLR - 1) / kLR, B * Hq);
+    const dim3 sg(B * Hq, (nb + kLR - 1) / kLR);
     gate_softmax_kernel<<<sg, kLThreads, ssmem, stream>>>(qt, kt, Hq, Hkv, nb, dg, 1.0f / sqrtf((float)dg), scores);
     return cudaGetLastError();
 }

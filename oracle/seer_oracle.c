@@ -50,7 +50,7 @@
 
 /* Number of blocks of a sequence of S tokens.  When S is not a multiple of 64
  * the last block holds the S - 64 (nb - 1) remaining tokens ([GATE Weakness
- * 3]: the pooling is padded / ceil-mode; the reading taken is that the last
+ * 4]: the pooling is padded / ceil-mode; the reading taken is that the last
  * block pools only its real tokens and that no query or key exists past S). */
 static int nblocks(int S) { return (S + SEER_ORACLE_BLOCK - 1) / SEER_ORACLE_BLOCK; }
 
