@@ -249,6 +249,71 @@ def pooled_map(q, k, v, scale: float | None = None, units=None):
     return o, A
 
 
+# --------------------------------------------------------------------------- decode
+# "SeerAttention-R: Sparse Attention Adaptation for Long Reasoning" (abstract):
+# the decode form keeps the self-distilled gate but drops query pooling, and
+# runs a block-sparse decoding kernel; "SeerAttention" rebuttal Weakness 4 on
+# decode: a per-Q-token AttnGate without pooling, on the same linear weights.
+# Reading: one new token per sequence at position L - 1 of a KV cache of L
+# tokens (its own k, v included), nb = ceil(L / 64).  Its query block is the
+# last one, i = nb - 1: the gate row is the prefill gate's row i with the
+# pooled query replaced by the token's own q, the mask row is the prefill
+# mask's row i, and the attention is the prefill attention of query row L - 1.
+# Each function below is exactly that: the pinned prefill functions applied
+# to arrays whose row i (or token L - 1) holds the decode data.
+def decode_gate_scores(q_tok, k, wq, wk, theta: float = 5e5, wq_head_stride=None, wk_head_stride=None,
+                       k_maxmin: bool = False) -> np.ndarray:
+    """Decode gate: q_tok bf16 [B,Hq,d] (no pooling), k bf16 [B,Hkv,L,d] -> f64 [B,Hq,nb]."""
+    q_tok, k = _u16(q_tok), _u16(k)
+    B, Hq, d = q_tok.shape
+    nb = -(-k.shape[2] // BLOCK)
+    dk = 2 * d if k_maxmin else d
+    dg = _u16(wq).shape[-1]
+    if wq_head_stride is None:
+        wq_head_stride = 0 if _u16(wq).ndim == 2 else d * dg
+    if wk_head_stride is None:
+        wk_head_stride = 0 if _u16(wk).ndim == 2 else dk * dg
+    kt = project_rope(pool_maxmin(k) if k_maxmin else pool_avg(k), wk, theta, head_stride=wk_head_stride)
+    xq = np.zeros((B, Hq, nb, d), np.float64)
+    xq[:, :, nb - 1] = (q_tok.astype(np.uint32) << 16).view(np.float32)     # bf16 bits -> value
+    qt = project_rope(xq, wq, theta, head_stride=wq_head_stride)
+    return block_softmax(qt, kt)[:, :, nb - 1, :].copy()
+
+
+def decode_mask(scores, mode: str, threshold: float = 0.0, k: int | None = None, force_first: bool = True,
+                force_diag: bool = True) -> np.ndarray:
+    """Decode mask row from f32 scores [B,Hq,nb] -> u8 [B,Hq,nb]; TopK keeps k
+    blocks (clamped to the forced set and to nb); the last block is the
+    token's own ("diagonal")."""
+    s = np.ascontiguousarray(scores, dtype=np.float32)
+    B, Hq, nb = s.shape
+    full = np.zeros((B, Hq, nb, nb), np.float32)
+    full[:, :, nb - 1] = s
+    kr = np.ones(nb, np.int32)
+    if mode == "topk":
+        kr[nb - 1] = int(k)
+    return block_mask(full, mode, threshold=threshold, k_row=kr, force_first=force_first,
+                      force_diag=force_diag)[:, :, nb - 1].copy()
+
+
+def decode_attention(q_tok, k, v, mask_row, scale: float | None = None):
+    """Decode attention of token L-1 over the active blocks of its mask row:
+    q_tok bf16 [B,Hq,d], k/v bf16 [B,Hkv,L,d], mask_row u8 [B,Hq,nb]
+    -> (o f64 [B,Hq,d], lse f64 [B,Hq])."""
+    q_tok, k, v = _u16(q_tok), _u16(k), _u16(v)
+    B, Hq, d = q_tok.shape
+    L = k.shape[2]
+    nb = -(-L // BLOCK)
+    Q = np.zeros((B, Hq, L, d), np.uint16)
+    Q[:, :, L - 1] = q_tok
+    mask = np.zeros((B, Hq, nb, nb), np.uint8)
+    mask[:, :, nb - 1] = np.asarray(mask_row, np.uint8)
+    units = np.array([(b, h, nb - 1) for b in range(B) for h in range(Hq)], np.int32)
+    o, lse = masked_attention(Q, k, v, mask, scale=scale, units=units)
+    r = L - 1 - BLOCK * (nb - 1)
+    return o[:, r].reshape(B, Hq, d), lse[:, r].reshape(B, Hq)
+
+
 def distill_loss(G, A):
     """Row-normalised target Ahat, per-row squared error and per-head mean
     (over causal block entries) of MSE(G, Ahat); G, A f32 [B,Hq,nb,nb]."""

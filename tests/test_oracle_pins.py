@@ -553,3 +553,82 @@ def test_ragged_pooled_map_brute_force(oracle):
         want = np.array([[p[a:b, c:e].max() if j <= i else 0.0 for j, (c, e) in enumerate(_blocks(S))]
                          for i, (a, b) in enumerate(_blocks(S))])
         np.testing.assert_allclose(A[h], want, rtol=1e-12, atol=0)
+
+
+# --------------------------------------------------------------------- decode
+def _rot(x, pos, theta, dg):
+    """Rotate-half RoPE at integer positions `pos` (broadcast over leading axes) via complex numbers."""
+    ang = np.asarray(pos)[..., None] * theta ** (-2.0 * np.arange(dg // 2) / dg)
+    z = (x[..., : dg // 2] + 1j * x[..., dg // 2:]) * np.exp(1j * ang)
+    return np.concatenate([z.real, z.imag], -1)
+
+
+@pytest.mark.parametrize("L,maxmin", [(5 * BLOCK + 20, False), (3 * BLOCK, True), (41, False)])
+def test_decode_gate_brute_force(oracle, L, maxmin):
+    """Decode gate: the token's own q (no pooling) projected and rotated at its
+    block (the last), against the pooled, projected, rotated K of every block."""
+    B, Hq, Hkv, d, dg, theta = 2, 4, 2, 16, 8, 1e3
+    qb = rand_bits((B, Hq, d), 120, scale=3.0)
+    kb = rand_bits((B, Hkv, L, d), 121, scale=3.0, shift=0.3)
+    dk = 2 * d if maxmin else d
+    wqb, wkb = rand_bits((Hq, d, dg), 122, scale=0.5), rand_bits((Hkv, dk, dg), 123, scale=0.5)
+    got = oracle.decode_gate_scores(qb, kb, wqb, wkb, theta=theta, k_maxmin=maxmin)
+    q, k = bits_to_f64(qb), bits_to_f64(kb)
+    blocks = _blocks(L)
+    nb = len(blocks)
+    if maxmin:
+        kp = np.stack([np.concatenate([k[:, :, a:b].max(2), k[:, :, a:b].min(2)], -1) for a, b in blocks], 2)
+    else:
+        kp = np.stack([k[:, :, a:b].mean(2) for a, b in blocks], 2)
+    kt = _rot(np.einsum("bhjd,hde->bhje", kp, bits_to_f64(wkb)), np.arange(nb), theta, dg)
+    qt = _rot(np.einsum("bhd,hde->bhe", q, bits_to_f64(wqb)), nb - 1, theta, dg)
+    lg = np.einsum("bhe,bhje->bhj", qt, np.repeat(kt, Hq // Hkv, axis=1)) / math.sqrt(dg)
+    e = np.exp(lg - lg.max(-1, keepdims=True))
+    assert got.shape == (B, Hq, nb)
+    np.testing.assert_allclose(got, e / e.sum(-1, keepdims=True), rtol=1e-11, atol=1e-15)
+    np.testing.assert_allclose(got.sum(-1), 1.0, rtol=1e-13)
+
+
+def test_decode_mask_brute_force(oracle):
+    B, Hq, nb = 2, 3, 37
+    s = rng(124).random((B, Hq, nb)).astype(np.float32)
+    s[0, 0, 5] = s[0, 0, 9] = s[0, 0, 20]            # ties go to the lower block
+    for k in (1, 2, 5, 11, nb, nb + 4):
+        got = oracle.decode_mask(s, "topk", k=k)
+        for b in range(B):
+            for h in range(Hq):
+                want = np.zeros(nb, np.uint8)
+                want[0] = want[nb - 1] = 1
+                rest = [j for j in sorted(range(1, nb - 1), key=lambda j: (-s[b, h, j], j))]
+                for j in rest[: max(0, min(k, nb) - 2)]:
+                    want[j] = 1
+                np.testing.assert_array_equal(got[b, h], want)
+    thr = np.float32(0.5)
+    got = oracle.decode_mask(s, "threshold", threshold=thr)
+    want = (s > thr).astype(np.uint8)
+    want[..., 0] = want[..., nb - 1] = 1
+    np.testing.assert_array_equal(got, want)
+
+
+@pytest.mark.parametrize("L", [7 * BLOCK + 13, 4 * BLOCK, 30])
+def test_decode_attention_brute_force(oracle, L):
+    B, Hq, Hkv, d = 1, 4, 2, 16
+    nb = len(_blocks(L))
+    qb = rand_bits((B, Hq, d), 125, scale=2.0)
+    kb, vb = rand_bits((B, Hkv, L, d), 126), rand_bits((B, Hkv, L, d), 127)
+    m = (rng(128).random((B, Hq, nb)) < 0.5).astype(np.uint8)
+    m[..., nb - 1] = 1
+    o, lse = oracle.decode_attention(qb, kb, vb, m, scale=0.3)
+    q, k, v = bits_to_f64(qb), bits_to_f64(kb), bits_to_f64(vb)
+    for h in range(Hq):
+        act = m[0, h][np.arange(L) // BLOCK].astype(bool)
+        s = np.where(act, k[0, h // 2] @ q[0, h] * 0.3, -np.inf)
+        p = np.exp(s - s.max())
+        np.testing.assert_allclose(o[0, h], p @ v[0, h // 2] / p.sum(), rtol=1e-10, atol=1e-12)
+        np.testing.assert_allclose(lse[0, h], s.max() + np.log(p.sum()), rtol=1e-12)
+    # every block active: plain softmax over all L keys (the token sees the whole cache)
+    o1, _ = oracle.decode_attention(qb, kb, vb, np.ones((B, Hq, nb), np.uint8), scale=0.3)
+    s = np.einsum("hcd,hd->hc", np.repeat(k[0], 2, axis=0), q[0]) * 0.3
+    p = np.exp(s - s.max(-1, keepdims=True))
+    np.testing.assert_allclose(o1[0], np.einsum("hc,hcd->hd", p, np.repeat(v[0], 2, axis=0)) / p.sum(-1, keepdims=True),
+                               rtol=1e-10, atol=1e-12)
