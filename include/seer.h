@@ -108,7 +108,9 @@ typedef struct seer_mask_params {
 enum {
     SEER_CALL_GATE_SCORES = 0,
     SEER_CALL_BLOCK_SPARSE_PREFILL = 1,
-    SEER_CALL_ATTN_POOLED_MAP = 2
+    SEER_CALL_ATTN_POOLED_MAP = 2,
+    SEER_CALL_DECODE_GATE_SCORES = 3,
+    SEER_CALL_BLOCK_SPARSE_DECODE = 4
 };
 
 /*
@@ -219,6 +221,51 @@ SEER_API seer_status seer_gate_scores_noalloc(const seer_shape *shape, const voi
  */
 SEER_API seer_status seer_distill_loss(const seer_shape *shape, const float *scores, const float *A,
                                        float *A_norm, float *loss_rows, float *loss, void *stream);
+
+/*
+ * Decode step ("SeerAttention-R: Sparse Attention Adaptation for Long
+ * Reasoning", abstract: the gate keeps its self-distilled design but drops
+ * query pooling, and a sparse decoding kernel reads only the selected KV
+ * blocks; "Learning Intrinsic Sparse Attention", rebuttal Weakness 4 on
+ * decode: a per-Q-token AttnGate without pooling on the same weights).
+ * One new token per sequence at position L - 1 of a KV cache of L tokens
+ * that already holds its k and v; shape->S = L, nb = ceil(L/64), and the
+ * token's block is the last one, i = nb - 1.
+ *
+ * seer_decode_gate_scores — the gate row of the token:
+ *   qt = RoPE_{nb-1}(q_tok @ Wq[h])          (the token's own q, no pooling)
+ *   Kt_j = RoPE_j(Kp_j @ Wk[h_kv])           (Kp as in seer_gate_scores)
+ *   scores[b,h,j] = softmax_j(qt . Kt_j / sqrt(d_gate)), j < nb.
+ * q_tok: bf16 [B,Hq,d]; k: bf16 [B,Hkv,L,d]; wq/wk and params as in
+ * seer_gate_scores; scores: fp32 [B,Hq,nb].  Workspace:
+ * seer_workspace_bytes(SEER_CALL_DECODE_GATE_SCORES, shape), 256-B aligned.
+ */
+SEER_API seer_status seer_decode_gate_scores(const seer_shape *shape, const void *q_tok, const void *k,
+                                             const void *wq, const void *wk, const seer_gate_params *gp,
+                                             float *scores, void *workspace, size_t ws_bytes, void *stream);
+
+/*
+ * seer_decode_block_mask — the mask row of the token: seer_block_mask's row
+ * i = nb - 1 (threshold or TopK with k from k_fixed, k_per_row[nb-1] or
+ * ceil(density * nb); block 0 and the last block forced as flagged).
+ * scores: fp32 [B,Hq,nb]; mask: u8 [B,Hq,nb], fully written.  No workspace.
+ */
+SEER_API seer_status seer_decode_block_mask(const seer_shape *shape, const float *scores,
+                                            const seer_mask_params *mp, uint8_t *mask, void *stream);
+
+/*
+ * seer_block_sparse_decode — attention of the token over the active blocks:
+ *   o[b,h] = sum_{c < L, mask[b,h,c/64]} softmax(q_tok . k_c * scale) v_c,
+ *   lse[b,h] = log sum exp (fp32, natural log; -inf and o = 0 when no block
+ *   is active).  scale <= 0 means 1/sqrt(d).
+ * q_tok: bf16 [B,Hq,d]; k/v: bf16 [B,Hkv,L,d]; mask: u8 [B,Hq,nb];
+ * o: bf16 [B,Hq,d]; lse: fp32 [B,Hq] or NULL.  Workspace:
+ * seer_workspace_bytes(SEER_CALL_BLOCK_SPARSE_DECODE, shape), 16-B aligned
+ * (split-K partials).
+ */
+SEER_API seer_status seer_block_sparse_decode(const seer_shape *shape, const void *q_tok, const void *k,
+                                              const void *v, const uint8_t *mask, float softmax_scale, void *o,
+                                              float *lse, void *workspace, size_t ws_bytes, void *stream);
 
 /* Workspace bytes a call needs for `shape` (0 for SEER_CALL_BLOCK_SPARSE_PREFILL).
  * Returns 0 and sets the last error for an invalid shape or call id. */

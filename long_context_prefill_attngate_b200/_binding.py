@@ -30,6 +30,8 @@ SEER_MASK_TOPK = 1
 SEER_CALL_GATE_SCORES = 0
 SEER_CALL_BLOCK_SPARSE_PREFILL = 1
 SEER_CALL_ATTN_POOLED_MAP = 2
+SEER_CALL_DECODE_GATE_SCORES = 3
+SEER_CALL_BLOCK_SPARSE_DECODE = 4
 
 BLOCK = 64
 
@@ -38,6 +40,7 @@ EXPORTS = (
     "seer_gate_scores", "seer_block_mask", "seer_compact_mask", "seer_block_sparse_prefill",
     "seer_attn_pooled_map", "seer_workspace_bytes", "seer_check_status", "seer_set_wait_timeout_ns",
     "seer_last_error", "seer_version", "seer_gate_scores_noalloc", "seer_distill_loss",
+    "seer_decode_gate_scores", "seer_decode_block_mask", "seer_block_sparse_decode",
 )
 
 
@@ -90,9 +93,13 @@ def lib() -> ctypes.CDLL:
             L.seer_distill_loss.argtypes = [SP, P, P, P, P, P, P]
             L.seer_block_sparse_prefill.argtypes = [SP, P, P, P, P, F, P, P, P, Z, P]
             L.seer_attn_pooled_map.argtypes = [SP, P, P, P, F, P, P, P, Z, P]
+            L.seer_decode_gate_scores.argtypes = [SP, P, P, P, P, ctypes.POINTER(seer_gate_params), P, P, Z, P]
+            L.seer_decode_block_mask.argtypes = [SP, P, ctypes.POINTER(seer_mask_params), P, P]
+            L.seer_block_sparse_decode.argtypes = [SP, P, P, P, P, F, P, P, P, Z, P]
             for fn in ("seer_gate_scores", "seer_gate_scores_noalloc", "seer_block_mask", "seer_compact_mask",
                        "seer_block_sparse_prefill", "seer_attn_pooled_map", "seer_check_status",
-                       "seer_distill_loss"):
+                       "seer_distill_loss", "seer_decode_gate_scores", "seer_decode_block_mask",
+                       "seer_block_sparse_decode"):
                 getattr(L, fn).restype = I
             L.seer_workspace_bytes.argtypes = [I, SP]
             L.seer_workspace_bytes.restype = Z
@@ -300,6 +307,76 @@ def seer_distill_loss(scores, A, want_norm: bool = False, stream=None, Hkv: int 
     _check(lib().seer_distill_loss(ctypes.byref(sh), _ptr(scores), _ptr(A), _ptr(an), _ptr(rows), _ptr(loss),
                                    _stream_ptr(stream)))
     return loss, rows, an
+
+
+# ------------------------------------------------------------------ decode step
+def _decode_shape(q_tok, k):
+    _need(q_tok.dim() == 3 and k.dim() == 4, "q_tok must be [B,Hq,d] and k [B,Hkv,L,d]")
+    B, Hq, d = q_tok.shape
+    _need(k.shape[0] == B and k.shape[3] == d, "q_tok / k shapes disagree")
+    return seer_shape(B, Hq, k.shape[1], k.shape[2], d)
+
+
+def seer_decode_gate_scores(q_tok, k, wq, wk, rope_theta: float = 5e5, scores=None, workspace=None, stream=None,
+                            wq_head_stride: int | None = None, wk_head_stride: int | None = None,
+                            k_maxmin: bool = False):
+    """Decode gate row fp32 [B,Hq,nb] of the token at position L-1 (see include/seer.h)."""
+    torch = _torch()
+    _need(q_tok.is_contiguous() and k.is_contiguous() and wq.is_contiguous() and wk.is_contiguous(),
+          "tensors must be contiguous")
+    _need(q_tok.dtype == k.dtype == wq.dtype == wk.dtype == torch.bfloat16, "q_tok, k, wq, wk must be bf16")
+    sh = _decode_shape(q_tok, k)
+    d, dg = sh.d, wq.shape[-1]
+    nb = -(-sh.S // BLOCK)
+    if wq_head_stride is None:
+        wq_head_stride = 0 if wq.dim() == 2 else d * dg
+    if wk_head_stride is None:
+        wk_head_stride = 0 if wk.dim() == 2 else (2 * d if k_maxmin else d) * dg
+    _need(wk.shape[-2] == (2 * d if k_maxmin else d) and wk.shape[-1] == dg, "wk shape does not match k pooling")
+    if scores is None:
+        scores = torch.empty((sh.B, sh.Hq, nb), dtype=torch.float32, device=q_tok.device)
+    workspace, wsb = _workspace(SEER_CALL_DECODE_GATE_SCORES, sh, q_tok.device, workspace)
+    gp = seer_gate_params(int(dg), float(rope_theta), int(wq_head_stride), int(wk_head_stride), int(bool(k_maxmin)))
+    _check(lib().seer_decode_gate_scores(ctypes.byref(sh), _ptr(q_tok), _ptr(k), _ptr(wq), _ptr(wk),
+                                         ctypes.byref(gp), _ptr(scores), _ptr(workspace), wsb, _stream_ptr(stream)))
+    return scores
+
+
+def seer_decode_block_mask(scores, mode: str = "topk", threshold: float = 0.0, density: float = 1.0,
+                           k_fixed: int = 0, force_first: bool = True, force_diag: bool = True, mask=None,
+                           stream=None):
+    """Decode mask row u8 [B,Hq,nb] from the gate row (threshold or TopK)."""
+    torch = _torch()
+    _need(scores.dtype == torch.float32 and scores.is_contiguous() and scores.dim() == 3,
+          "scores must be contiguous fp32 [B,Hq,nb]")
+    B, Hq, nb = scores.shape
+    sh = seer_shape(B, Hq, 1, nb * BLOCK, 64)
+    if mask is None:
+        mask = torch.empty((B, Hq, nb), dtype=torch.uint8, device=scores.device)
+    m = {"threshold": SEER_MASK_THRESHOLD, "topk": SEER_MASK_TOPK}[mode]
+    mp = seer_mask_params(m, float(threshold), float(density), int(k_fixed), None,
+                          int(bool(force_first)), int(bool(force_diag)))
+    _check(lib().seer_decode_block_mask(ctypes.byref(sh), _ptr(scores), ctypes.byref(mp), _ptr(mask),
+                                        _stream_ptr(stream)))
+    return mask
+
+
+def seer_block_sparse_decode(q_tok, k, v, mask, softmax_scale: float = 0.0, o=None, lse=None,
+                             return_lse: bool = False, workspace=None, stream=None):
+    """Attention of the token at position L-1 over its active KV blocks; returns o [B,Hq,d] bf16."""
+    torch = _torch()
+    _need(all(t.is_contiguous() for t in (q_tok, k, v, mask)), "tensors must be contiguous")
+    _need(q_tok.dtype == k.dtype == v.dtype == torch.bfloat16 and mask.dtype == torch.uint8, "bf16 q/k/v, u8 mask")
+    sh = _decode_shape(q_tok, k)
+    if o is None:
+        o = torch.empty_like(q_tok)
+    if return_lse and lse is None:
+        lse = torch.empty((sh.B, sh.Hq), dtype=torch.float32, device=q_tok.device)
+    workspace, wsb = _workspace(SEER_CALL_BLOCK_SPARSE_DECODE, sh, q_tok.device, workspace)
+    _check(lib().seer_block_sparse_decode(ctypes.byref(sh), _ptr(q_tok), _ptr(k), _ptr(v), _ptr(mask),
+                                          float(softmax_scale), _ptr(o), _ptr(lse), _ptr(workspace), wsb,
+                                          _stream_ptr(stream)))
+    return (o, lse) if (return_lse or lse is not None) else o
 
 
 def topk_counts(density: float, nb: int, force_first: bool = True, force_diag: bool = True) -> list[int]:

@@ -172,21 +172,26 @@ size_t seer_workspace_bytes(int which_call, const seer_shape *shape)
         return 0;
     case SEER_CALL_ATTN_POOLED_MAP:
         return sizeof(float) * (size_t)kMaxAttnCtas * nb * 128;
+    case SEER_CALL_DECODE_GATE_SCORES:
+        return gate_workspace_bytes(shape->B, shape->Hq, shape->Hkv, shape->S, shape->d, 256, true);
+    case SEER_CALL_BLOCK_SPARSE_DECODE:
+        return sizeof(float) * (size_t)shape->B * shape->Hq * kMaxDecodeSplits * (shape->d + 2);
     default:
         fail(SEER_ERR_INVALID_ARG, "unknown call id %d", which_call);
         return 0;
     }
 }
 
-seer_status seer_gate_scores(const seer_shape *shape, const void *q, const void *k, const void *wq, const void *wk,
-                             const seer_gate_params *gp, float *scores, void *workspace, size_t ws_bytes,
-                             void *stream)
+// Argument checks shared by the prefill and decode gates.
+static seer_status check_gate_args(const char *name, const seer_shape *shape, const void *q, const void *k,
+                                   const void *wq, const void *wk, const seer_gate_params *gp, const float *scores,
+                                   void *workspace, size_t ws_bytes)
 {
     seer_status st = check_shape(shape);
     if (st != SEER_OK)
         return st;
     if (gp == nullptr || q == nullptr || k == nullptr || wq == nullptr || wk == nullptr || scores == nullptr)
-        return fail(SEER_ERR_INVALID_ARG, "seer_gate_scores: NULL argument");
+        return fail(SEER_ERR_INVALID_ARG, "%s: NULL argument", name);
     if (gp->d_gate < 2 || gp->d_gate > 256 || (gp->d_gate & 1))
         return fail(SEER_ERR_UNSUPPORTED, "d_gate %d must be even and in [2, 256]", gp->d_gate);
     if (!(gp->rope_theta > 0.f) || !std::isfinite(gp->rope_theta))
@@ -206,9 +211,20 @@ seer_status seer_gate_scores(const seer_shape *shape, const void *q, const void 
     const size_t need =
         gate_workspace_bytes(shape->B, shape->Hq, shape->Hkv, shape->S, shape->d, gp->d_gate, maxmin);
     if (workspace == nullptr || ws_bytes < need)
-        return fail(SEER_ERR_WORKSPACE, "seer_gate_scores needs %zu workspace bytes, got %zu", need, ws_bytes);
+        return fail(SEER_ERR_WORKSPACE, "%s needs %zu workspace bytes, got %zu", name, need, ws_bytes);
     if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
         return fail(SEER_ERR_WORKSPACE, "workspace must be 256-byte aligned");
+    return SEER_OK;
+}
+
+seer_status seer_gate_scores(const seer_shape *shape, const void *q, const void *k, const void *wq, const void *wk,
+                             const seer_gate_params *gp, float *scores, void *workspace, size_t ws_bytes,
+                             void *stream)
+{
+    const seer_status st = check_gate_args("seer_gate_scores", shape, q, k, wq, wk, gp, scores, workspace, ws_bytes);
+    if (st != SEER_OK)
+        return st;
+    const bool maxmin = gp->k_pooling == SEER_KPOOL_MAXMIN;
     const cudaError_t e = launch_gate(shape->B, shape->Hq, shape->Hkv, shape->S, shape->d, gp->d_gate,
                                       gp->rope_theta, maxmin, q, k, wq, gp->wq_head_stride, wk, gp->wk_head_stride,
                                       scores, workspace, static_cast<cudaStream_t>(stream));
@@ -386,6 +402,76 @@ seer_status seer_check_status(void *stream)
             return fail(SEER_ERR_TIMEOUT, "a device-side wait ran out");
         return fail(SEER_ERR_DEVICE, "device-side check failed (code %d)", v);
     }
+    return ok();
+}
+
+// ---------------------------------------------------------------- decode step
+seer_status seer_decode_gate_scores(const seer_shape *shape, const void *q_tok, const void *k, const void *wq,
+                                    const void *wk, const seer_gate_params *gp, float *scores, void *workspace,
+                                    size_t ws_bytes, void *stream)
+{
+    const seer_status st =
+        check_gate_args("seer_decode_gate_scores", shape, q_tok, k, wq, wk, gp, scores, workspace, ws_bytes);
+    if (st != SEER_OK)
+        return st;
+    if (num_blocks(shape->S) * sizeof(float) + 1024 > 227 * 1024)
+        return fail(SEER_ERR_UNSUPPORTED, "seer_decode_gate_scores: nb = %d too large", num_blocks(shape->S));
+    const cudaError_t e = launch_decode_gate(shape->B, shape->Hq, shape->Hkv, shape->S, shape->d, gp->d_gate,
+                                             gp->rope_theta, gp->k_pooling == SEER_KPOOL_MAXMIN, q_tok, k, wq,
+                                             gp->wq_head_stride, wk, gp->wk_head_stride, scores, workspace,
+                                             static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess)
+        return cuda_fail(e, "seer_decode_gate_scores launch");
+    return ok();
+}
+
+seer_status seer_decode_block_mask(const seer_shape *shape, const float *scores, const seer_mask_params *mp,
+                                   uint8_t *mask, void *stream)
+{
+    seer_status st = check_shape(shape);
+    if (st != SEER_OK)
+        return st;
+    if (mp == nullptr || scores == nullptr || mask == nullptr)
+        return fail(SEER_ERR_INVALID_ARG, "seer_decode_block_mask: NULL argument");
+    if (mp->mode != SEER_MASK_THRESHOLD && mp->mode != SEER_MASK_TOPK)
+        return fail(SEER_ERR_INVALID_ARG, "unknown mask mode %d", mp->mode);
+    if (mp->mode == SEER_MASK_TOPK && mp->k_per_row == nullptr && mp->k_fixed <= 0 &&
+        !(std::isfinite(mp->density) && mp->density >= 0.0))
+        return fail(SEER_ERR_INVALID_ARG, "TopK density must be finite and >= 0");
+    if (mp->mode == SEER_MASK_THRESHOLD && std::isnan(mp->threshold))
+        return fail(SEER_ERR_INVALID_ARG, "threshold is NaN");
+    const int nb = num_blocks(shape->S);
+    const cudaError_t e = launch_mask_rows(shape->B, shape->Hq, nb, 1, nb - 1, scores, mp->mode, mp->threshold,
+                                           mp->density, mp->k_fixed, mp->k_per_row, mp->force_first ? 1 : 0,
+                                           mp->force_diag ? 1 : 0, mask, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess)
+        return cuda_fail(e, "seer_decode_block_mask launch");
+    return ok();
+}
+
+seer_status seer_block_sparse_decode(const seer_shape *shape, const void *q_tok, const void *k, const void *v,
+                                     const uint8_t *mask, float softmax_scale, void *o, float *lse, void *workspace,
+                                     size_t ws_bytes, void *stream)
+{
+    seer_status st = attention_common("seer_block_sparse_decode", shape, q_tok, k, v, o);
+    if (st != SEER_OK)
+        return st;
+    if (mask == nullptr)
+        return fail(SEER_ERR_INVALID_ARG, "seer_block_sparse_decode: NULL mask");
+    if (std::isnan(softmax_scale) || std::isinf(softmax_scale))
+        return fail(SEER_ERR_INVALID_ARG, "softmax_scale must be finite");
+    const size_t need = seer_workspace_bytes(SEER_CALL_BLOCK_SPARSE_DECODE, shape);
+    if (workspace == nullptr || ws_bytes < need)
+        return fail(SEER_ERR_WORKSPACE, "seer_block_sparse_decode needs %zu workspace bytes, got %zu", need,
+                    ws_bytes);
+    if ((reinterpret_cast<uintptr_t>(workspace) & 15u) != 0)
+        return fail(SEER_ERR_WORKSPACE, "workspace must be 16-byte aligned");
+    const float scale = softmax_scale > 0.f ? softmax_scale : 1.0f / sqrtf((float)shape->d);
+    const cudaError_t e =
+        launch_decode(shape->B, shape->Hq, shape->Hkv, shape->S, shape->d, scale * 1.4426950408889634f, q_tok, k, v,
+                      mask, o, lse, static_cast<float *>(workspace), static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess)
+        return cuda_fail(e, "seer_block_sparse_decode launch");
     return ok();
 }
 

@@ -1,0 +1,258 @@
+// seer_decode.cu — block-sparse attention of one new token per sequence over
+// its KV cache: the decode step of "SeerAttention-R: Sparse Attention
+// Adaptation for Long Reasoning" (the gate without query pooling selects KV
+// blocks; a sparse decoding kernel reads only those).
+//
+// o[b,h] = sum over keys c < L in active blocks of softmax(q . k_c * scale) v_c
+// for the token at position L - 1 (every cached key is at or before it).
+//
+// Decode reads each active K/V block once and does 2 x 64 x d flops per block
+// with them: it is bound by HBM (and L2, for blocks the heads of a GQA group
+// share), so this is a CUDA-core kernel sized for memory parallelism, not a
+// tensor-core one:
+//  * split-K over the active blocks (flash-decoding): CTA (split s, head bh)
+//    takes the active blocks whose rank in the mask row is s mod nsplit, keeps
+//    an online softmax and writes (o, m, l) partials; a second kernel merges
+//    the splits and normalises.
+//  * per block: 128 threads = 64 keys x 2 halves of d for the scores (16-byte
+//    loads of K rows), then D/2 dim pairs x (128 / (D/2)) key groups for
+//    P V (coalesced bf16x2 loads of V rows).
+//  * many small CTAs per SM keep many blocks in flight.
+#include <cuda_bf16.h>
+
+#include "seer_internal.h"
+
+namespace seer {
+
+namespace {
+
+constexpr int kDT = 128;             // threads per CTA
+constexpr int kChunk = kDT;          // mask entries ranked per pass
+
+__device__ __forceinline__ float exp2_approx(float x)
+{
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+template <int D>
+__global__ void __launch_bounds__(kDT)
+    decode_attn_kernel(const __nv_bfloat16 *__restrict__ q_tok, const __nv_bfloat16 *__restrict__ k,
+                       const __nv_bfloat16 *__restrict__ v, const uint8_t *__restrict__ mask, int Hq, int Hkv, int L,
+                       int nb, float scale_log2, int nsplit, float *__restrict__ part)
+{
+    constexpr int DH = D / 2;            // dims per thread in the score dot
+    constexpr int NP = D / 2;            // dim pairs
+    constexpr int KG = kDT / NP;         // key groups in P V (2 for d = 128, 4 for d = 64)
+    constexpr int KPG = 64 / KG;         // keys per group
+    __shared__ int s_list[kChunk];
+    __shared__ int s_wsum[kDT / 32];
+    __shared__ float s_red[kDT / 32];
+    __shared__ float s_p[64];
+    __shared__ float s_o[KG][D];
+    const int split = blockIdx.x;
+    const long long bh = blockIdx.y;
+    const int b = (int)(bh / Hq), h = (int)(bh % Hq);
+    const int kvh = h / (Hq / Hkv);
+    const uint8_t *mrow = mask + bh * nb;
+    const __nv_bfloat16 *kb = k + ((long long)b * Hkv + kvh) * L * D;
+    const __nv_bfloat16 *vb = v + ((long long)b * Hkv + kvh) * L * D;
+    const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
+    const int kr = t >> 1, hf = t & 1;            // score role: key, half of d
+    const int dp = t % NP, kg = t / NP;           // P V role: dim pair, key group
+
+    float qv[DH];
+    {
+        const uint4 *qr = reinterpret_cast<const uint4 *>(q_tok + bh * D + hf * DH);
+#pragma unroll
+        for (int c = 0; c < DH / 8; ++c) {
+            const uint4 u = qr[c];
+            const __nv_bfloat162 *p2 = reinterpret_cast<const __nv_bfloat162 *>(&u);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const float2 f = __bfloat1622float2(p2[e]);
+                qv[8 * c + 2 * e] = f.x;
+                qv[8 * c + 2 * e + 1] = f.y;
+            }
+        }
+    }
+    float m = -INFINITY, l = 0.f, o0 = 0.f, o1 = 0.f;
+    int rank_base = 0;
+    for (int j0 = 0; j0 < nb; j0 += kChunk) {
+        // Rank the active blocks of this chunk; keep those with rank = split (mod nsplit).
+        const int j = j0 + t;
+        const int a = (j < nb && mrow[j] != 0) ? 1 : 0;
+        const unsigned bal = __ballot_sync(0xffffffffu, a);
+        if (lane == 0)
+            s_wsum[warp] = __popc(bal);
+        __syncthreads();
+        int before = 0, total = 0;
+#pragma unroll
+        for (int w = 0; w < kDT / 32; ++w) {
+            before += w < warp ? s_wsum[w] : 0;
+            total += s_wsum[w];
+        }
+        const int rank = rank_base + before + __popc(bal & ((1u << lane) - 1u));
+        // this split's entries of the chunk, in rank order
+        const int first = (rank_base % nsplit <= split) ? rank_base + (split - rank_base % nsplit)
+                                                        : rank_base + nsplit - (rank_base % nsplit - split);
+        if (a && (rank % nsplit) == split)
+            s_list[(rank - first) / nsplit] = j;
+        const int mine = (first < rank_base + total) ? (rank_base + total - 1 - first) / nsplit + 1 : 0;
+        rank_base += total;
+        __syncthreads();
+        for (int e = 0; e < mine; ++e) {
+            const int jb = s_list[e];
+            // ---- scores of the block's 64 keys
+            const int c = jb * 64 + kr;
+            float s = 0.f;
+            if (c < L) {
+                const uint4 *kp = reinterpret_cast<const uint4 *>(kb + (long long)c * D + hf * DH);
+#pragma unroll
+                for (int cc = 0; cc < DH / 8; ++cc) {
+                    const uint4 u = __ldg(kp + cc);
+                    const __nv_bfloat162 *p2 = reinterpret_cast<const __nv_bfloat162 *>(&u);
+#pragma unroll
+                    for (int ee = 0; ee < 4; ++ee) {
+                        const float2 f = __bfloat1622float2(p2[ee]);
+                        s = fmaf(qv[8 * cc + 2 * ee], f.x, fmaf(qv[8 * cc + 2 * ee + 1], f.y, s));
+                    }
+                }
+            }
+            s += __shfl_xor_sync(0xffffffffu, s, 1);
+            s = (c < L) ? s * scale_log2 : -INFINITY;
+            float wm = s;
+#pragma unroll
+            for (int off = 16; off >= 1; off >>= 1)
+                wm = fmaxf(wm, __shfl_xor_sync(0xffffffffu, wm, off));
+            if (lane == 0)
+                s_red[warp] = wm;
+            __syncthreads();
+            float bm = s_red[0];
+#pragma unroll
+            for (int w = 1; w < kDT / 32; ++w)
+                bm = fmaxf(bm, s_red[w]);
+            const float m_new = fmaxf(m, bm);        // finite: key 0 of every block exists
+            const float alpha = exp2_approx(m - m_new);
+            const float p = exp2_approx(s - m_new);
+            if (hf == 0)
+                s_p[kr] = p;
+            __syncthreads();
+            // ---- P V for this thread's dim pair over its key group
+            float a0 = 0.f, a1 = 0.f, ls = 0.f;
+#pragma unroll 4
+            for (int q = 0; q < KPG; ++q) {
+                const int key = kg * KPG + q;
+                const int cc = jb * 64 + key;
+                const float pk = s_p[key];
+                ls += pk;
+                if (cc < L) {
+                    const float2 f = __bfloat1622float2(
+                        *reinterpret_cast<const __nv_bfloat162 *>(vb + (long long)cc * D + 2 * dp));
+                    a0 = fmaf(pk, f.x, a0);
+                    a1 = fmaf(pk, f.y, a1);
+                }
+            }
+            o0 = o0 * alpha + a0;
+            o1 = o1 * alpha + a1;
+            l = l * alpha + ls;                      // this key group's share of the row sum
+            m = m_new;
+            __syncthreads();                         // s_p / s_red are reused by the next block
+        }
+    }
+    // Merge the key groups: o and l summed over groups (same m everywhere).
+    s_o[kg][2 * dp] = o0;
+    s_o[kg][2 * dp + 1] = o1;
+    if (dp == 0)
+        s_p[kg] = l;
+    __syncthreads();
+    float *out = part + (bh * nsplit + split) * (D + 2);
+    for (int d = t; d < D; d += kDT) {
+        float acc = 0.f;
+#pragma unroll
+        for (int g = 0; g < KG; ++g)
+            acc += s_o[g][d];
+        out[d] = acc;
+    }
+    if (t == 0) {
+        float lt = 0.f;
+#pragma unroll
+        for (int g = 0; g < KG; ++g)
+            lt += s_p[g];
+        out[D] = m;
+        out[D + 1] = lt;
+    }
+}
+
+// Merge the splits of one head: weights 2^(m_s - M), O = sum w o / sum w l.
+template <int D>
+__global__ void __launch_bounds__(D)
+    decode_combine_kernel(const float *__restrict__ part, int nsplit, __nv_bfloat16 *__restrict__ o,
+                          float *__restrict__ lse)
+{
+    const long long bh = blockIdx.x;
+    const float *pp = part + bh * nsplit * (D + 2);
+    float M = -INFINITY;
+    for (int s = 0; s < nsplit; ++s)
+        M = fmaxf(M, pp[s * (D + 2) + D]);
+    float acc = 0.f, lt = 0.f;
+    if (M != -INFINITY) {
+        for (int s = 0; s < nsplit; ++s) {
+            const float ms = pp[s * (D + 2) + D];
+            const float w = ms == -INFINITY ? 0.f : exp2_approx(ms - M);
+            acc = fmaf(w, pp[s * (D + 2) + threadIdx.x], acc);
+            lt = fmaf(w, pp[s * (D + 2) + D + 1], lt);
+        }
+    }
+    const bool has = lt > 0.f;
+    o[bh * D + threadIdx.x] = __float2bfloat16(has ? acc / lt : 0.f);
+    if (lse != nullptr && threadIdx.x == 0)
+        lse[bh] = has ? (M + __log2f(lt)) * 0.69314718055994530942f : -INFINITY;
+}
+
+} // namespace
+
+int decode_splits(int B, int Hq, int nb)
+{
+    static int sms = 0;
+    if (sms == 0) {
+        int dev = 0, v = 0;
+        if (cudaGetDevice(&dev) == cudaSuccess &&
+            cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && v > 0)
+            sms = v;
+        else
+            sms = 148;
+    }
+    const long long heads = (long long)B * Hq;
+    long long s = (8LL * sms + heads - 1) / heads;     // about eight CTAs per SM
+    if (s > kMaxDecodeSplits)
+        s = kMaxDecodeSplits;
+    if (s > nb)
+        s = nb;
+    return (int)(s < 1 ? 1 : s);
+}
+
+cudaError_t launch_decode(int B, int Hq, int Hkv, int L, int d, float scale_log2, const void *q_tok, const void *k,
+                          const void *v, const uint8_t *mask, void *o, float *lse, float *part, cudaStream_t stream)
+{
+    const int nb = num_blocks(L);
+    const int ns = decode_splits(B, Hq, nb);
+    const dim3 grid(ns, B * Hq);
+    const auto *qb = static_cast<const __nv_bfloat16 *>(q_tok);
+    const auto *kb = static_cast<const __nv_bfloat16 *>(k);
+    const auto *vb = static_cast<const __nv_bfloat16 *>(v);
+    auto *ob = static_cast<__nv_bfloat16 *>(o);
+    if (d == 128) {
+        decode_attn_kernel<128><<<grid, kDT, 0, stream>>>(qb, kb, vb, mask, Hq, Hkv, L, nb, scale_log2, ns, part);
+        decode_combine_kernel<128><<<B * Hq, 128, 0, stream>>>(part, ns, ob, lse);
+    } else if (d == 64) {
+        decode_attn_kernel<64><<<grid, kDT, 0, stream>>>(qb, kb, vb, mask, Hq, Hkv, L, nb, scale_log2, ns, part);
+        decode_combine_kernel<64><<<B * Hq, 64, 0, stream>>>(part, ns, ob, lse);
+    } else {
+        return cudaErrorInvalidValue;
+    }
+    return cudaGetLastError();
+}
+
+} // namespace seer

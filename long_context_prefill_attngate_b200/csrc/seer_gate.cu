@@ -103,14 +103,14 @@ constexpr int kProjRows = 64;
 constexpr int kProjThreads = 256;      // 16 x 16: rows ty + 16a, rotation pairs tx + 16b
 constexpr int kPStride = 4;            // padding (floats) of the shared rows
 
-// out[bh, i, :] = RoPE_i( xp[bh, i, :] @ W[h] ) for 64 blocks i of one head.
+// out[bh, i, :] = RoPE_{pos0+i}( xp[bh, i, :] @ W[h] ) for 64 rows i of one head.
 // Each thread owns 4 rows x 4 rotation pairs (t, t + dg/2), so both halves
 // of a pair are in its registers when the rotation is applied.  Angles
 // i * theta^(-2t/dg): frequencies in double once per CTA, angle formed and
 // reduced modulo 2*pi in double, the reduced angle through fp32 sincosf.
 __global__ void __launch_bounds__(kProjThreads)
     project_rope_kernel(const float *__restrict__ xp, int H, int nb, int d, const __nv_bfloat16 *__restrict__ w,
-                        long long w_stride, int dg, double theta, float *__restrict__ out)
+                        long long w_stride, int dg, double theta, int pos0, float *__restrict__ out)
 {
     extern __shared__ float4 psm4[];
     const int xs = d + kPStride;
@@ -177,7 +177,7 @@ __global__ void __launch_bounds__(kProjThreads)
                 const int t = t0 + tx + 16 * b;
                 if (t >= half)
                     continue;
-                const double ang = (double)i * sfreq[t];
+                const double ang = (double)(pos0 + i) * sfreq[t];
                 const double red = ang - rint(ang * (1.0 / kTwoPi)) * kTwoPi;
                 float sn, cs;
                 sincosf((float)red, &sn, &cs);
@@ -326,6 +326,76 @@ __global__ void __launch_bounds__(kLThreads)
     }
 }
 
+// Decode: the new token's q (bf16 [B*Hq, d]) as fp32 rows for the projection.
+__global__ void q_to_f32_kernel(const __nv_bfloat16 *__restrict__ q, long long n, float *__restrict__ out)
+{
+    for (long long e = (long long)blockIdx.x * blockDim.x + threadIdx.x; e < n; e += (long long)gridDim.x * blockDim.x)
+        out[e] = __bfloat162float(q[e]);
+}
+
+constexpr int kDecThreads = 256;
+
+// Decode gate row: scores[bh, j] = softmax_j(qt[bh] . kt[b, h/g, j] / sqrt(dg))
+// over every block j < nb (the token sits in the last block).  One CTA per
+// (b, h): logits into shared memory (nb floats), then max / sum / normalise.
+__global__ void __launch_bounds__(kDecThreads)
+    decode_gate_kernel(const float *__restrict__ qt, const float *__restrict__ kt, int Hq, int Hkv, int nb, int dg,
+                       float scale, float *__restrict__ scores)
+{
+    extern __shared__ float dsm[];
+    float *sq = dsm;                 // dg
+    float *sl = dsm + dg;            // nb
+    __shared__ float red[kDecThreads / 32];
+    const int bh = blockIdx.x;
+    const int b = bh / Hq, h = bh % Hq;
+    const float *kb = kt + (long long)(b * Hkv + h / (Hq / Hkv)) * nb * dg;
+    for (int c = threadIdx.x; c < dg; c += kDecThreads)
+        sq[c] = qt[(long long)bh * dg + c];
+    __syncthreads();
+    float mx = -INFINITY;
+    for (int j = threadIdx.x; j < nb; j += kDecThreads) {
+        const float4 *kr = reinterpret_cast<const float4 *>(kb + (long long)j * dg);
+        float acc = 0.f;
+        for (int c4 = 0; c4 < dg / 4; ++c4) {
+            const float4 kv = __ldg(kr + c4);
+            acc = fmaf(sq[4 * c4], kv.x,
+                       fmaf(sq[4 * c4 + 1], kv.y, fmaf(sq[4 * c4 + 2], kv.z, fmaf(sq[4 * c4 + 3], kv.w, acc))));
+        }
+        acc *= scale;
+        sl[j] = acc;
+        mx = fmaxf(mx, acc);
+    }
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+#pragma unroll
+    for (int off = 16; off >= 1; off >>= 1)
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+    if (lane == 0)
+        red[warp] = mx;
+    __syncthreads();
+    mx = red[0];
+    for (int w = 1; w < kDecThreads / 32; ++w)
+        mx = fmaxf(mx, red[w]);
+    __syncthreads();
+    float sum = 0.f;
+    for (int j = threadIdx.x; j < nb; j += kDecThreads) {
+        const float e = expf(sl[j] - mx);
+        sl[j] = e;
+        sum += e;
+    }
+#pragma unroll
+    for (int off = 16; off >= 1; off >>= 1)
+        sum += __shfl_xor_sync(0xffffffffu, sum, off);
+    if (lane == 0)
+        red[warp] = sum;
+    __syncthreads();
+    sum = 0.f;
+    for (int w = 0; w < kDecThreads / 32; ++w)
+        sum += red[w];
+    const float inv = 1.0f / sum;
+    for (int j = threadIdx.x; j < nb; j += kDecThreads)
+        scores[(long long)bh * nb + j] = sl[j] * inv;
+}
+
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 } // namespace
@@ -386,10 +456,10 @@ cudaError_t launch_gate(int B, int Hq, int Hkv, int S, int d, int dg, float thet
     const dim3 pg_k((nb + kProjRows - 1) / kProjRows, B * Hkv);
     project_rope_kernel<<<pg_q, kProjThreads, psmem_q, stream>>>(qp, Hq, nb, d,
                                                                static_cast<const __nv_bfloat16 *>(wq), wq_stride,
-                                                               dg, (double)theta, qt);
+                                                               dg, (double)theta, 0, qt);
     project_rope_kernel<<<pg_k, kProjThreads, psmem, stream>>>(kp, Hkv, nb, dk,
                                                                static_cast<const __nv_bfloat16 *>(wk), wk_stride,
-                                                               dg, (double)theta, kt);
+                                                               dg, (double)theta, 0, kt);
     e = cudaGetLastError();
     if (e != cudaSuccess)
         return e;
@@ -399,6 +469,69 @@ cudaError_t launch_gate(int B, int Hq, int Hkv, int S, int d, int dg, float thet
         return e;
     const dim3 sg(B * Hq, (nb + kLR - 1) / kLR);
     gate_softmax_kernel<<<sg, kLThreads, ssmem, stream>>>(qt, kt, Hq, Hkv, nb, dg, 1.0f / sqrtf((float)dg), scores);
+    return cudaGetLastError();
+}
+
+} // namespace seer
+
+namespace seer {
+
+// Decode gate ("SeerAttention-R": the gate without query pooling): the K side
+// is the prefill gate's (pooled K of the L-token cache, projected, block
+// RoPE); the token's q is projected and rotated at its block, nb - 1.  The
+// workspace layout is the prefill gate's (its Q regions hold the q rows).
+cudaError_t launch_decode_gate(int B, int Hq, int Hkv, int L, int d, int dg, float theta, bool k_maxmin,
+                               const void *q_tok, const void *k, const void *wq, long long wq_stride, const void *wk,
+                               long long wk_stride, float *scores, void *ws, cudaStream_t stream)
+{
+    const int nb = num_blocks(L);
+    const int dk = k_maxmin ? 2 * d : d;
+    char *p = static_cast<char *>(ws);
+    float *qp = reinterpret_cast<float *>(p);
+    p += align256(sizeof(float) * B * Hq * (size_t)nb * d);
+    float *kp = reinterpret_cast<float *>(p);
+    p += align256(sizeof(float) * B * Hkv * (size_t)nb * dk);
+    float *qt = reinterpret_cast<float *>(p);
+    p += align256(sizeof(float) * B * Hq * (size_t)nb * dg);
+    float *kt = reinterpret_cast<float *>(p);
+
+    const auto *kb = static_cast<const __nv_bfloat16 *>(k);
+    const unsigned gk = (unsigned)((long long)B * Hkv * nb);
+    if (d == 128) {
+        if (k_maxmin)
+            pool_kernel<128, true><<<gk, kPoolThreads, 0, stream>>>(kb, L, nb, kp);
+        else
+            pool_kernel<128><<<gk, kPoolThreads, 0, stream>>>(kb, L, nb, kp);
+    } else {
+        if (k_maxmin)
+            pool_kernel<64, true><<<gk, kPoolThreads, 0, stream>>>(kb, L, nb, kp);
+        else
+            pool_kernel<64><<<gk, kPoolThreads, 0, stream>>>(kb, L, nb, kp);
+    }
+    const long long nq = (long long)B * Hq * d;
+    q_to_f32_kernel<<<(unsigned)((nq + 255) / 256), 256, 0, stream>>>(static_cast<const __nv_bfloat16 *>(q_tok), nq,
+                                                                       qp);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess)
+        return e;
+    const size_t psmem = gate_projection_smem(dk, dg);
+    e = cudaFuncSetAttribute(project_rope_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)psmem);
+    if (e != cudaSuccess)
+        return e;
+    // q: one row per head at position nb - 1; K: every block.
+    project_rope_kernel<<<dim3(1, B * Hq), kProjThreads, gate_projection_smem(d, dg), stream>>>(
+        qp, Hq, 1, d, static_cast<const __nv_bfloat16 *>(wq), wq_stride, dg, (double)theta, nb - 1, qt);
+    project_rope_kernel<<<dim3((nb + kProjRows - 1) / kProjRows, B * Hkv), kProjThreads, psmem, stream>>>(
+        kp, Hkv, nb, dk, static_cast<const __nv_bfloat16 *>(wk), wk_stride, dg, (double)theta, 0, kt);
+    e = cudaGetLastError();
+    if (e != cudaSuccess)
+        return e;
+    const size_t dsmem = sizeof(float) * (size_t)(dg + nb);
+    e = cudaFuncSetAttribute(decode_gate_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dsmem);
+    if (e != cudaSuccess)
+        return e;
+    decode_gate_kernel<<<B * Hq, kDecThreads, dsmem, stream>>>(qt, kt, Hq, Hkv, nb, dg, 1.0f / sqrtf((float)dg),
+                                                                scores);
     return cudaGetLastError();
 }
 

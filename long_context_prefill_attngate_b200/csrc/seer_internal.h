@@ -43,11 +43,23 @@ cudaError_t launch_gate(int B, int Hq, int Hkv, int S, int d, int dg, float thet
                         float *scores, void *ws, cudaStream_t stream);
 size_t gate_workspace_bytes(int B, int Hq, int Hkv, int S, int d, int dg, bool k_maxmin);
 size_t gate_projection_smem(int d_in, int dg);
+cudaError_t launch_decode_gate(int B, int Hq, int Hkv, int L, int d, int dg, float theta, bool k_maxmin,
+                               const void *q_tok, const void *k, const void *wq, long long wq_stride, const void *wk,
+                               long long wk_stride, float *scores, void *ws, cudaStream_t stream);
+
+// Block-sparse decode attention (seer_decode.cu).
+constexpr int kMaxDecodeSplits = 64;
+int decode_splits(int B, int Hq, int nb);
+cudaError_t launch_decode(int B, int Hq, int Hkv, int L, int d, float scale_log2, const void *q_tok, const void *k,
+                          const void *v, const uint8_t *mask, void *o, float *lse, float *part, cudaStream_t stream);
 
 // Mask / compaction kernels (seer_mask.cu).
 cudaError_t launch_mask(int B, int Hq, int nb, const float *scores, int mode, float threshold,
                         double density, int k_fixed, const int32_t *k_per_row, int force_first,
                         int force_diag, uint8_t *mask, cudaStream_t stream);
+cudaError_t launch_mask_rows(int B, int Hq, int nb, int R, int i0, const float *scores, int mode, float threshold,
+                             double density, int k_fixed, const int32_t *k_per_row, int ff, int fd, uint8_t *mask,
+                             cudaStream_t stream);
 cudaError_t launch_compact(int B, int Hq, int nb, const uint8_t *mask, int32_t *lists, int32_t *counts,
                            cudaStream_t stream);
 

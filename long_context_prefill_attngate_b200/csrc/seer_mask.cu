@@ -23,13 +23,13 @@ namespace {
 constexpr int kThrThreads = 256;
 
 __global__ void __launch_bounds__(kThrThreads)
-    threshold_kernel(const float *__restrict__ scores, long long total, int nb, float thr, int ff, int fd,
-                     uint8_t *__restrict__ mask)
+    threshold_kernel(const float *__restrict__ scores, long long total, int nb, int R, int i0, float thr, int ff,
+                     int fd, uint8_t *__restrict__ mask)
 {
     for (long long e = (long long)blockIdx.x * kThrThreads + threadIdx.x; e < total;
          e += (long long)gridDim.x * kThrThreads) {
         const int j = (int)(e % nb);
-        const int i = (int)((e / nb) % nb);
+        const int i = i0 + (int)((e / nb) % R);
         uint8_t m = 0;
         if (j <= i)
             m = (scores[e] > thr) || (ff && j == 0) || (fd && j == i);
@@ -85,7 +85,7 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int *sbuf, int *total
 
 // One CTA per row (b, h, i).
 __global__ void __launch_bounds__(kTopThreads)
-    topk_kernel(const float *__restrict__ scores, int nb, double density, int k_fixed,
+    topk_kernel(const float *__restrict__ scores, int nb, int R, int i0, double density, int k_fixed,
                 const int32_t *__restrict__ k_per_row, int ff, int fd, uint8_t *__restrict__ mask)
 {
     extern __shared__ uint32_t keys[];        // nb entries
@@ -94,7 +94,7 @@ __global__ void __launch_bounds__(kTopThreads)
     __shared__ uint32_t s_prefix;
     __shared__ int s_remaining;
     const long long row = blockIdx.x;
-    const int i = (int)(row % nb);
+    const int i = i0 + (int)(row % R);
     const float *srow = scores + row * nb;
     uint8_t *mrow = mask + row * nb;
     const int n = i + 1;
@@ -204,14 +204,14 @@ __device__ __forceinline__ int row_k(int i, double density, int k_fixed, const i
 // Absent entries (j > i) hold key 0, below every real key.
 template <int PER>
 __global__ void __launch_bounds__(256)
-    topk_warp_kernel(const float *__restrict__ scores, long long rows, int nb, double density, int k_fixed,
-                     const int32_t *__restrict__ k_per_row, int ff, int fd, uint8_t *__restrict__ mask)
+    topk_warp_kernel(const float *__restrict__ scores, long long rows, int nb, int R, int i0, double density,
+                     int k_fixed, const int32_t *__restrict__ k_per_row, int ff, int fd, uint8_t *__restrict__ mask)
 {
     const long long row = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
     if (row >= rows)
         return;
     const int lane = threadIdx.x & 31;
-    const int i = (int)(row % nb);
+    const int i = i0 + (int)(row % R);
     const int n = i + 1;
     const float *srow = scores + row * nb;
     uint8_t *mrow = mask + row * nb;
@@ -296,32 +296,48 @@ __global__ void __launch_bounds__(256)
 cudaError_t launch_mask(int B, int Hq, int nb, const float *scores, int mode, float threshold, double density,
                         int k_fixed, const int32_t *k_per_row, int ff, int fd, uint8_t *mask, cudaStream_t stream)
 {
-    const long long rows = (long long)B * Hq * nb;
+    return launch_mask_rows(B, Hq, nb, nb, 0, scores, mode, threshold, density, k_fixed, k_per_row, ff, fd, mask,
+                            stream);
+}
+
+// R score rows of nb entries per head, row r holding causal row i0 + r (the
+// prefill square: R = nb, i0 = 0; a decode step: R = 1, i0 = nb - 1).
+cudaError_t launch_mask_rows(int B, int Hq, int nb, int R, int i0, const float *scores, int mode, float threshold,
+                             double density, int k_fixed, const int32_t *k_per_row, int ff, int fd, uint8_t *mask,
+                             cudaStream_t stream)
+{
+    const long long rows = (long long)B * Hq * R;
     if (mode == 0) {
         const long long total = rows * nb;
         long long blocks = (total + kThrThreads - 1) / kThrThreads;
         if (blocks > 148LL * 64)
             blocks = 148LL * 64;
-        threshold_kernel<<<(unsigned)blocks, kThrThreads, 0, stream>>>(scores, total, nb, threshold, ff, fd, mask);
+        threshold_kernel<<<(unsigned)blocks, kThrThreads, 0, stream>>>(scores, total, nb, R, i0, threshold, ff, fd,
+                                                                       mask);
         return cudaGetLastError();
     }
     if (nb <= 1024) {
         const unsigned grid = (unsigned)((rows + 7) / 8);
         if (nb <= 128)
-            topk_warp_kernel<4><<<grid, 256, 0, stream>>>(scores, rows, nb, density, k_fixed, k_per_row, ff, fd, mask);
+            topk_warp_kernel<4><<<grid, 256, 0, stream>>>(scores, rows, nb, R, i0, density, k_fixed, k_per_row, ff,
+                                                               fd, mask);
         else if (nb <= 256)
-            topk_warp_kernel<8><<<grid, 256, 0, stream>>>(scores, rows, nb, density, k_fixed, k_per_row, ff, fd, mask);
+            topk_warp_kernel<8><<<grid, 256, 0, stream>>>(scores, rows, nb, R, i0, density, k_fixed, k_per_row, ff,
+                                                               fd, mask);
         else if (nb <= 512)
-            topk_warp_kernel<16><<<grid, 256, 0, stream>>>(scores, rows, nb, density, k_fixed, k_per_row, ff, fd, mask);
+            topk_warp_kernel<16><<<grid, 256, 0, stream>>>(scores, rows, nb, R, i0, density, k_fixed, k_per_row, ff,
+                                                               fd, mask);
         else
-            topk_warp_kernel<32><<<grid, 256, 0, stream>>>(scores, rows, nb, density, k_fixed, k_per_row, ff, fd, mask);
+            topk_warp_kernel<32><<<grid, 256, 0, stream>>>(scores, rows, nb, R, i0, density, k_fixed, k_per_row, ff,
+                                                               fd, mask);
         return cudaGetLastError();
     }
     const size_t smem = sizeof(uint32_t) * (size_t)nb;
     cudaError_t e = cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess)
         return e;
-    topk_kernel<<<(unsigned)rows, kTopThreads, smem, stream>>>(scores, nb, density, k_fixed, k_per_row, ff, fd, mask);
+    topk_kernel<<<(unsigned)rows, kTopThreads, smem, stream>>>(scores, nb, R, i0, density, k_fixed, k_per_row, ff, fd,
+                                                               mask);
     return cudaGetLastError();
 }
 
