@@ -21,6 +21,7 @@
 #include <cuda_bf16.h>
 
 #include "seer_internal.h"
+#include "seer_ptx.cuh"
 
 namespace seer {
 
@@ -185,6 +186,231 @@ __global__ void __launch_bounds__(kDT)
     }
 }
 
+
+// ---------------------------------------------------------------------------
+// GQA-group form (g = Hq/Hkv <= 8): one CTA per (kv head, split) serves all g
+// query heads, so each K/V block crosses HBM -> SM once for the group.  The
+// CTA walks the union of the heads' active blocks (a head that did not select
+// a block gets p = 0 there and keeps its running max and sum: exact).  K and V
+// blocks are staged in shared memory with cp.async, two blocks ahead.
+constexpr int kGT = 256;             // threads
+constexpr int kGMax = 8;             // heads per group served by this form
+
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src, int src_bytes)
+{
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
+template <int D>
+__global__ void __launch_bounds__(kGT)
+    decode_gqa_kernel(const __nv_bfloat16 *__restrict__ q_tok, const __nv_bfloat16 *__restrict__ k,
+                      const __nv_bfloat16 *__restrict__ v, const uint8_t *__restrict__ mask, int Hq, int Hkv, int L,
+                      int nb, float scale_log2, int nsplit, float *__restrict__ part)
+{
+    constexpr int RS = D + 8;                     // padded smem row (bf16): conflict-free 16-B reads
+    constexpr int DQ = D / 4;                     // dims per thread in the score dot (4 dim quarters)
+    constexpr int DPT = D / 32;                   // output dims per thread in P V
+    extern __shared__ __align__(16) uint8_t gsm[];
+    __nv_bfloat16 *sk = reinterpret_cast<__nv_bfloat16 *>(gsm);            // [2][64][RS]
+    __nv_bfloat16 *sv = sk + 2 * 64 * RS;                                  // [2][64][RS]
+    float *sq = reinterpret_cast<float *>(sv + 2 * 64 * RS);               // [kGMax][D]
+    float *sred = sq + kGMax * D;                                          // [4][kGMax][64]
+    float *sp = sred + 4 * kGMax * 64;                                     // [kGMax][64]
+    float *salpha = sp + kGMax * 64;                                       // [kGMax]
+    int *slist = reinterpret_cast<int *>(salpha + kGMax);                  // [kChunk] block | head bits << 16
+    int *swsum = slist + kGT;                                              // [kGT / 32]
+    const int split = blockIdx.x;
+    const int bk = blockIdx.y;                                             // b * Hkv + kvh
+    const int b = bk / Hkv, kvh = bk % Hkv;
+    const int g = Hq / Hkv;
+    const int h0 = kvh * g;
+    const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
+    const __nv_bfloat16 *kb = k + (long long)bk * L * D;
+    const __nv_bfloat16 *vb = v + (long long)bk * L * D;
+    const uint8_t *mbase = mask + ((long long)b * Hq + h0) * nb;
+    for (int e = t; e < g * D; e += kGT)
+        sq[e] = __bfloat162float(q_tok[((long long)b * Hq + h0) * D + e]);
+
+    // per-head online state: warp w < g owns head w's (m, l); every thread's
+    // P V accumulators belong to head (t / 32)
+    float m_h = -INFINITY, l_h = 0.f;
+    float acc[DPT];
+#pragma unroll
+    for (int i = 0; i < DPT; ++i)
+        acc[i] = 0.f;
+
+    auto issue = [&](int stage, int jb) {
+        // 64 rows of K and of V, D bf16 each: 64 * D / 8 16-byte pieces per tensor
+        const uint32_t dk = smem_u32(sk + stage * 64 * RS), dv = smem_u32(sv + stage * 64 * RS);
+        for (int e = t; e < 64 * D / 8; e += kGT) {
+            const int r = e / (D / 8), c8 = e % (D / 8);
+            const int row = jb * 64 + r;
+            const bool ok = row < L;
+            const long long off = (long long)(ok ? row : 0) * D + c8 * 8;
+            cp_async16(dk + (uint32_t)(r * RS + c8 * 8) * 2, kb + off, ok ? 16 : 0);
+            cp_async16(dv + (uint32_t)(r * RS + c8 * 8) * 2, vb + off, ok ? 16 : 0);
+        }
+    };
+
+    int rank_base = 0;
+    for (int j0 = 0; j0 < nb; j0 += kGT) {
+        // union of the group's mask rows over this chunk, ranked; this split keeps rank = split (mod nsplit)
+        const int j = j0 + t;
+        int bitsj = 0;
+        if (j < nb)
+            for (int hh = 0; hh < g; ++hh)
+                bitsj |= (mbase[(long long)hh * nb + j] != 0) << hh;
+        const int a = bitsj != 0;
+        const unsigned bal = __ballot_sync(0xffffffffu, a);
+        if (lane == 0)
+            swsum[warp] = __popc(bal);
+        __syncthreads();
+        int before = 0, total = 0;
+#pragma unroll
+        for (int w = 0; w < kGT / 32; ++w) {
+            before += w < warp ? swsum[w] : 0;
+            total += swsum[w];
+        }
+        const int rank = rank_base + before + __popc(bal & ((1u << lane) - 1u));
+        const int r0 = rank_base % nsplit;
+        const int first = rank_base + (split >= r0 ? split - r0 : nsplit - (r0 - split));
+        if (a && (rank % nsplit) == split)
+            slist[(rank - first) / nsplit] = j | (bitsj << 16);
+        const int mine = (first < rank_base + total) ? (rank_base + total - 1 - first) / nsplit + 1 : 0;
+        rank_base += total;
+        __syncthreads();
+        if (mine > 0)
+            issue(0, slist[0] & 0xFFFF);
+        cp_async_commit();
+        if (mine > 1)
+            issue(1, slist[1] & 0xFFFF);
+        cp_async_commit();
+        for (int e = 0; e < mine; ++e) {
+            const int st = e & 1;
+            const int jb = slist[e] & 0xFFFF;
+            const int hbits = slist[e] >> 16;
+            cp_async_wait<1>();                       // this block's group is complete
+            __syncthreads();
+            // ---- scores: thread = (key c, dim quarter dq), all g heads
+            {
+                const int c = t & 63, dq = t >> 6;
+                const __nv_bfloat16 *kr = sk + (st * 64 + c) * RS + dq * DQ;
+                float kf[DQ];
+#pragma unroll
+                for (int i = 0; i < DQ / 8; ++i) {
+                    const uint4 u = *reinterpret_cast<const uint4 *>(kr + 8 * i);
+                    const __nv_bfloat162 *p2 = reinterpret_cast<const __nv_bfloat162 *>(&u);
+#pragma unroll
+                    for (int e2 = 0; e2 < 4; ++e2) {
+                        const float2 f = __bfloat1622float2(p2[e2]);
+                        kf[8 * i + 2 * e2] = f.x;
+                        kf[8 * i + 2 * e2 + 1] = f.y;
+                    }
+                }
+                for (int hh = 0; hh < g; ++hh) {
+                    const float *qh = sq + hh * D + dq * DQ;
+                    float s = 0.f;
+#pragma unroll
+                    for (int i = 0; i < DQ; ++i)
+                        s = fmaf(qh[i], kf[i], s);
+                    sred[(dq * kGMax + hh) * 64 + c] = s;
+                }
+            }
+            __syncthreads();
+            // ---- per-head online softmax: warp hh handles head hh
+            if (warp < g) {
+                const int hh = warp;
+                const bool act = (hbits >> hh) & 1;
+                float s0 = -INFINITY, s1 = -INFINITY;
+                if (act) {
+                    const int c0 = lane, c1 = lane + 32;
+                    s0 = (sred[hh * 64 + c0] + sred[(kGMax + hh) * 64 + c0] + sred[(2 * kGMax + hh) * 64 + c0] +
+                          sred[(3 * kGMax + hh) * 64 + c0]) * scale_log2;
+                    s1 = (sred[hh * 64 + c1] + sred[(kGMax + hh) * 64 + c1] + sred[(2 * kGMax + hh) * 64 + c1] +
+                          sred[(3 * kGMax + hh) * 64 + c1]) * scale_log2;
+                    if (jb * 64 + c0 >= L)
+                        s0 = -INFINITY;
+                    if (jb * 64 + c1 >= L)
+                        s1 = -INFINITY;
+                }
+                float bm = fmaxf(s0, s1);
+#pragma unroll
+                for (int off = 16; off >= 1; off >>= 1)
+                    bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, off));
+                const float m_new = act ? fmaxf(m_h, bm) : m_h;
+                const float alpha = act ? exp2_approx(m_h - m_new) : 1.0f;
+                const float p0 = act ? exp2_approx(s0 - m_new) : 0.f;
+                const float p1 = act ? exp2_approx(s1 - m_new) : 0.f;
+                float ps = p0 + p1;
+#pragma unroll
+                for (int off = 16; off >= 1; off >>= 1)
+                    ps += __shfl_xor_sync(0xffffffffu, ps, off);
+                sp[hh * 64 + lane] = p0;
+                sp[hh * 64 + lane + 32] = p1;
+                if (lane == 0)
+                    salpha[hh] = alpha;
+                l_h = l_h * alpha + ps;
+                m_h = m_new;
+            }
+            __syncthreads();
+            // ---- P V: warp hh accumulates head hh's output dims
+            if (warp < g) {
+                const int hh = warp;
+                const float alpha = salpha[hh];
+#pragma unroll
+                for (int i = 0; i < DPT; ++i)
+                    acc[i] *= alpha;
+                const __nv_bfloat16 *vr = sv + st * 64 * RS + lane * DPT;
+#pragma unroll 8
+                for (int c = 0; c < 64; ++c) {
+                    const float pc = sp[hh * 64 + c];
+                    if (DPT == 4) {
+                        const uint2 u = *reinterpret_cast<const uint2 *>(vr + c * RS);
+                        const float2 f0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&u.x));
+                        const float2 f1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&u.y));
+                        acc[0] = fmaf(pc, f0.x, acc[0]);
+                        acc[1] = fmaf(pc, f0.y, acc[1]);
+                        acc[2 % DPT] = fmaf(pc, f1.x, acc[2 % DPT]);
+                        acc[3 % DPT] = fmaf(pc, f1.y, acc[3 % DPT]);
+                    } else {
+                        const float2 f0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(vr + c * RS));
+                        acc[0] = fmaf(pc, f0.x, acc[0]);
+                        acc[1 % DPT] = fmaf(pc, f0.y, acc[1 % DPT]);
+                    }
+                }
+            }
+            __syncthreads();                          // stage st is free again
+            if (e + 2 < mine)
+                issue(st, slist[e + 2] & 0xFFFF);
+            cp_async_commit();
+        }
+        cp_async_wait<0>();
+        __syncthreads();
+    }
+    // ---- partials of the g heads for this split
+    if (warp < g) {
+        const int hh = warp;
+        float *out = part + (((long long)b * Hq + h0 + hh) * nsplit + split) * (D + 2);
+#pragma unroll
+        for (int i = 0; i < DPT; ++i)
+            out[lane * DPT + i] = acc[i];
+        if (lane == 0) {
+            out[D] = m_h;
+            out[D + 1] = l_h;
+        }
+    }
+}
+
+size_t gqa_smem_bytes(int D)
+{
+    return (size_t)2 * 2 * 64 * (D + 8) * 2 + sizeof(float) * ((size_t)kGMax * D + 4 * kGMax * 64 + kGMax * 64 +
+                                                                  kGMax) +
+           sizeof(int) * (kGT + kGT / 32);
+}
+
 // Merge the splits of one head: weights 2^(m_s - M), O = sum w o / sum w l.
 template <int D>
 __global__ void __launch_bounds__(D)
@@ -215,6 +441,13 @@ __global__ void __launch_bounds__(D)
 
 int decode_splits(int B, int Hq, int nb)
 {
+    return decode_splits_for(B, Hq, nb, 8);
+}
+
+// Splits so that about `per_sm` CTAs run per SM over `units` (heads, or KV
+// heads for the group form); at most kMaxDecodeSplits and nb.
+int decode_splits_for(int B, int units_per_b, int nb, int per_sm)
+{
     static int sms = 0;
     if (sms == 0) {
         int dev = 0, v = 0;
@@ -224,8 +457,8 @@ int decode_splits(int B, int Hq, int nb)
         else
             sms = 148;
     }
-    const long long heads = (long long)B * Hq;
-    long long s = (8LL * sms + heads - 1) / heads;     // about eight CTAs per SM
+    const long long heads = (long long)B * units_per_b;
+    long long s = ((long long)per_sm * sms + heads - 1) / heads;
     if (s > kMaxDecodeSplits)
         s = kMaxDecodeSplits;
     if (s > nb)
@@ -237,9 +470,34 @@ cudaError_t launch_decode(int B, int Hq, int Hkv, int L, int d, float scale_log2
                           const void *v, const uint8_t *mask, void *o, float *lse, float *part, cudaStream_t stream)
 {
     const int nb = num_blocks(L);
+    const int g = Hq / Hkv;
+    const auto *qb = static_cast<const __nv_bfloat16 *>(q_tok);
+    if (g <= kGMax && (d == 128 || d == 64)) {
+        // group form: one CTA per (KV head, split); split count = the per-head merge's
+        const int ns = decode_splits_for(B, Hkv, nb, 3);
+        const size_t smem = gqa_smem_bytes(d);
+        const dim3 grid(ns, B * Hkv);
+        auto *ob = static_cast<__nv_bfloat16 *>(o);
+        const auto *kb = static_cast<const __nv_bfloat16 *>(k);
+        const auto *vb = static_cast<const __nv_bfloat16 *>(v);
+        cudaError_t e;
+        if (d == 128) {
+            e = cudaFuncSetAttribute(decode_gqa_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+            if (e != cudaSuccess)
+                return e;
+            decode_gqa_kernel<128><<<grid, kGT, smem, stream>>>(qb, kb, vb, mask, Hq, Hkv, L, nb, scale_log2, ns, part);
+            decode_combine_kernel<128><<<B * Hq, 128, 0, stream>>>(part, ns, ob, lse);
+        } else {
+            e = cudaFuncSetAttribute(decode_gqa_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+            if (e != cudaSuccess)
+                return e;
+            decode_gqa_kernel<64><<<grid, kGT, smem, stream>>>(qb, kb, vb, mask, Hq, Hkv, L, nb, scale_log2, ns, part);
+            decode_combine_kernel<64><<<B * Hq, 64, 0, stream>>>(part, ns, ob, lse);
+        }
+        return cudaGetLastError();
+    }
     const int ns = decode_splits(B, Hq, nb);
     const dim3 grid(ns, B * Hq);
-    const auto *qb = static_cast<const __nv_bfloat16 *>(q_tok);
     const auto *kb = static_cast<const __nv_bfloat16 *>(k);
     const auto *vb = static_cast<const __nv_bfloat16 *>(v);
     auto *ob = static_cast<__nv_bfloat16 *>(o);

@@ -50,6 +50,7 @@ cudaError_t launch_decode_gate(int B, int Hq, int Hkv, int L, int d, int dg, flo
 // Block-sparse decode attention (seer_decode.cu).
 constexpr int kMaxDecodeSplits = 64;
 int decode_splits(int B, int Hq, int nb);
+int decode_splits_for(int B, int units_per_b, int nb, int per_sm);
 cudaError_t launch_decode(int B, int Hq, int Hkv, int L, int d, float scale_log2, const void *q_tok, const void *k,
                           const void *v, const uint8_t *mask, void *o, float *lse, float *part, cudaStream_t stream);
 

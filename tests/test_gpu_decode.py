@@ -102,6 +102,7 @@ def test_decode_mask_bit_exact(oracle, L):
     (1, 5, 1, 64 * 33 + 1, 128, 0.3),          # a one-token last block, g = 5
     (1, 4, 2, 50, 128, 1.0),                  # shorter than one block
     (1, 6, 2, 2048, 128, 1.0),                # dense decode
+    (1, 16, 1, 1500, 64, 0.4),                # g = 16: the per-head form (groups above 8)
 ])
 def test_decode_attention_parity(oracle, B, Hq, Hkv, L, d, p):
     w, q, k, v, wq, wk = decode_inputs(B, Hq, Hkv, L, d, 128, 321 + L)
