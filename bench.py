@@ -299,6 +299,44 @@ def run_gpu(args, world, rank, local):
                                   "frac_of_hbm_peak": round(byt / (ms * 1e-3) / 1e9 / pk["hbm_gbs"], 4)}
         del A, mws, om
 
+    # ---------------- decode step of the last token on the same cache (SeerAttention-R form)
+    decode = None
+    if not args.no_decode:
+        q_tok = q[:, :, -1].contiguous()
+        dws = torch.empty(seer.seer_workspace_bytes(seer.SEER_CALL_DECODE_GATE_SCORES, sh), dtype=torch.uint8,
+                          device=dev)
+        aws = torch.empty(seer.seer_workspace_bytes(seer.SEER_CALL_BLOCK_SPARSE_DECODE, sh), dtype=torch.uint8,
+                          device=dev)
+        ds = seer.seer_decode_gate_scores(q_tok, k, wq, wk, rope_theta=w.rope_theta, workspace=dws)
+        dm = seer.seer_decode_block_mask(ds, "topk", density=args.density)
+        do = seer.seer_block_sparse_decode(q_tok, k, v, dm, workspace=aws)
+        tg, tm, ta = [], [], []
+        for _ in range(10):
+            flush.zero_()
+            ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+            ev[0].record(stream)
+            seer.seer_decode_gate_scores(q_tok, k, wq, wk, rope_theta=w.rope_theta, scores=ds, workspace=dws)
+            ev[1].record(stream)
+            seer.seer_decode_block_mask(ds, "topk", density=args.density, mask=dm)
+            ev[2].record(stream)
+            seer.seer_block_sparse_decode(q_tok, k, v, dm, o=do, workspace=aws)
+            ev[3].record(stream)
+            torch.cuda.synchronize()
+            tg.append(ev[0].elapsed_time(ev[1]))
+            tm.append(ev[1].elapsed_time(ev[2]))
+            ta.append(ev[2].elapsed_time(ev[3]))
+        seer.seer_check_status()
+        g = w.Hq // w.Hkv
+        union = int(dm.view(w.B, w.Hkv, g, nb).amax(2).sum().item())      # (KV head, block) pairs read
+        kv_bytes = union * 64 * w.d * 2 * 2
+        ms_a = statistics.median(ta)
+        decode = {"cache_tokens": w.S, "batch": w.B, "density": round(float(dm.float().mean().item()), 4),
+                  "gate_us": round(statistics.median(tg) * 1e3, 1), "mask_us": round(statistics.median(tm) * 1e3, 1),
+                  "attention_us": round(ms_a * 1e3, 1), "kv_bytes": kv_bytes,
+                  "attention_gbs": round(kv_bytes / (ms_a * 1e-3) / 1e9, 1),
+                  "frac_of_hbm_peak": round(kv_bytes / (ms_a * 1e-3) / 1e9 / pk["hbm_gbs"], 4)}
+        del dws, aws
+
     # ---------------- e2e: pinned host inputs -> C ABI -> host output, per step
     hq, hk, hv = (x[n].pin_memory() for n in ("q", "k", "v"))
     hwq, hwk = x["wq"].pin_memory(), x["wk"].pin_memory()
@@ -365,7 +403,7 @@ def run_gpu(args, world, rank, local):
                      "frac_of_sustained": round(attn_tflops / pk["bf16_tflops_sustained"], 4),
                      "kernel": "attn_kernel<128,false> (seer_block_sparse_prefill)",
                      "algorithmic_flops_per_launch": flops},
-        "density_sweep": sweep, "pooled_map": pooled,
+        "density_sweep": sweep, "pooled_map": pooled, "decode": decode,
         "e2e": {"value": round(e2e_value, 2), "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 3)},
         "gpu_launches": launches_per_step * args.steps,
@@ -466,6 +504,7 @@ def main():
     ap.add_argument("--density", type=float, default=0.1)
     ap.add_argument("--no-sweep", action="store_true")
     ap.add_argument("--no-map", action="store_true")
+    ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--ref-units", type=int, default=16)
