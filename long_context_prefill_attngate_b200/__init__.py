@@ -19,4 +19,6 @@ from ._binding import (  # noqa: F401
     seer_version, seer_workspace_bytes, shape_of, topk_counts,
 )
 
+from .pipeline import HostPrefill  # noqa: F401,E402
+
 __version__ = "0.1.0"

@@ -473,3 +473,26 @@ def test_distill_loss(oracle, name):
         _, Ao = oracle.pooled_map(bits(x["q"]), bits(x["k"]), bits(x["v"]))
         _, _, heads_o = oracle.distill_loss(Go.astype(np.float32), Ao.reshape(Go.shape).astype(np.float32))
         check_rel(loss.cpu().numpy(), heads_o, "loss (oracle chain)")
+
+
+# ------------------------------------------------------------------ host-memory pipeline
+@pytest.mark.parametrize("B,Hq,Hkv,S,d", [(1, 8, 2, 4096, 128), (2, 4, 1, 2000, 64)])
+def test_host_prefill_matches_whole_layer_calls(oracle, B, Hq, Hkv, S, d):
+    """Group-by-group processing with overlapped copies gives the same bits as
+    one whole-layer call of each entry point."""
+    w = syn.custom("hostpipe", B, Hq, Hkv, S, d, number=401 + S)
+    x = syn.make_inputs(w)
+    hq, hk, hv, hwq, hwk = (x[n].pin_memory() for n in ("q", "k", "v", "wq", "wk"))
+    ho = torch.empty(hq.shape, dtype=torch.bfloat16).pin_memory()
+    hp = seer.HostPrefill(B, Hq, Hkv, S, d, w.d_gate)
+    for _ in range(2):                    # the second call reuses the buffers
+        ho.zero_()
+        hp.run(hq, hk, hv, hwq, hwk, ho, density=0.2, rope_theta=w.rope_theta)
+        torch.cuda.synchronize()
+    seer.seer_check_status()
+    s = seer.seer_gate_scores(dev(x["q"]), dev(x["k"]), dev(x["wq"]), dev(x["wk"]), rope_theta=w.rope_theta)
+    m = seer.seer_block_mask(s, "topk", density=0.2, Hkv=Hkv, d=d)
+    o = seer.seer_block_sparse_prefill(dev(x["q"]), dev(x["k"]), dev(x["v"]), m)
+    torch.cuda.synchronize()
+    assert torch.equal(hp.mask.cpu(), m.cpu())
+    assert torch.equal(ho, o.cpu())
