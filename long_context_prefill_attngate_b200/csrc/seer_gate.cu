@@ -99,12 +99,13 @@ __global__ void __launch_bounds__(kPoolThreads) pool_kernel(const __nv_bfloat16 
     }
 }
 
-constexpr int kProjRows = 64;
+constexpr int kProjRows = 64;               // query/key blocks per CTA (16 and 32 measured no faster)
+constexpr int kPA = kProjRows / 16;         // rows per thread
 constexpr int kProjThreads = 256;      // 16 x 16: rows ty + 16a, rotation pairs tx + 16b
 constexpr int kPStride = 4;            // padding (floats) of the shared rows
 
-// out[bh, i, :] = RoPE_{pos0+i}( xp[bh, i, :] @ W[h] ) for 64 rows i of one head.
-// Each thread owns 4 rows x 4 rotation pairs (t, t + dg/2), so both halves
+// out[bh, i, :] = RoPE_{pos0+i}( xp[bh, i, :] @ W[h] ) for kProjRows rows i of one
+// head.  Each thread owns kPA rows x 4 rotation pairs (t, t + dg/2), so both halves
 // of a pair are in its registers when the rotation is applied.  Angles
 // i * theta^(-2t/dg): frequencies in double once per CTA, angle formed and
 // reduced modulo 2*pi in double, the reduced angle through fp32 sincosf.
@@ -123,8 +124,23 @@ __global__ void __launch_bounds__(kProjThreads)
     const int rows = min(kProjRows, nb - i0);
     const int half = dg / 2;
     const __nv_bfloat16 *wh = w + (long long)h * w_stride;
-    for (int e = threadIdx.x; e < d * dg; e += kProjThreads)
-        sw[e] = __bfloat162float(wh[e]);
+    // W as 16-byte pieces (8 bf16) when this head's weights start 16-byte aligned
+    if ((reinterpret_cast<uintptr_t>(wh) & 15) == 0 && ((d * dg) & 7) == 0) {
+        const uint4 *w4 = reinterpret_cast<const uint4 *>(wh);
+        for (int e = threadIdx.x; e < d * dg / 8; e += kProjThreads) {
+            const uint4 u = __ldg(w4 + e);
+            const __nv_bfloat162 *p2 = reinterpret_cast<const __nv_bfloat162 *>(&u);
+#pragma unroll
+            for (int k2 = 0; k2 < 4; ++k2) {
+                const float2 f = __bfloat1622float2(p2[k2]);
+                sw[8 * e + 2 * k2] = f.x;
+                sw[8 * e + 2 * k2 + 1] = f.y;
+            }
+        }
+    } else {
+        for (int e = threadIdx.x; e < d * dg; e += kProjThreads)
+            sw[e] = __bfloat162float(wh[e]);
+    }
     const float *xb = xp + ((long long)bh * nb + i0) * d;
     for (int e = threadIdx.x; e < kProjRows * d; e += kProjThreads) {
         const int r = e / d, c = e % d;
@@ -136,9 +152,9 @@ __global__ void __launch_bounds__(kProjThreads)
     constexpr double kTwoPi = 6.283185307179586476925286766559;
     const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
     for (int t0 = 0; t0 < half; t0 += 64) {
-        float y0[4][4], y1[4][4];
+        float y0[kPA][4], y1[kPA][4];
 #pragma unroll
-        for (int a = 0; a < 4; ++a)
+        for (int a = 0; a < kPA; ++a)
 #pragma unroll
             for (int b = 0; b < 4; ++b)
                 y0[a][b] = y1[a][b] = 0.f;
@@ -148,9 +164,9 @@ __global__ void __launch_bounds__(kProjThreads)
             tcol[b] = min(t0 + tx + 16 * b, half - 1);
 #pragma unroll 2
         for (int c = 0; c < d; ++c) {
-            float xv[4], w0[4], w1[4];
+            float xv[kPA], w0[4], w1[4];
 #pragma unroll
-            for (int a = 0; a < 4; ++a)
+            for (int a = 0; a < kPA; ++a)
                 xv[a] = sx[(ty + 16 * a) * xs + c];
 #pragma unroll
             for (int b = 0; b < 4; ++b) {
@@ -158,7 +174,7 @@ __global__ void __launch_bounds__(kProjThreads)
                 w1[b] = sw[c * dg + tcol[b] + half];
             }
 #pragma unroll
-            for (int a = 0; a < 4; ++a)
+            for (int a = 0; a < kPA; ++a)
 #pragma unroll
                 for (int b = 0; b < 4; ++b) {
                     y0[a][b] = fmaf(xv[a], w0[b], y0[a][b]);
@@ -166,7 +182,7 @@ __global__ void __launch_bounds__(kProjThreads)
                 }
         }
 #pragma unroll
-        for (int a = 0; a < 4; ++a) {
+        for (int a = 0; a < kPA; ++a) {
             const int r = ty + 16 * a;
             if (r >= rows)
                 continue;
@@ -188,7 +204,7 @@ __global__ void __launch_bounds__(kProjThreads)
     }
 }
 
-constexpr int kLR = 32;              // query blocks per CTA
+constexpr int kLR = 32;              // query blocks per CTA (16, 64, 128 measured slower)
 constexpr int kLA = kLR / 16;        // query rows per thread
 constexpr int kLC = 64;              // key blocks per tile
 constexpr int kLThreads = 256;       // 16 x 16: rows ty + 16a, columns tx + 16b
