@@ -348,25 +348,27 @@ def run_gpu(args, world, rank, local):
     # The library's host-memory entry (long_context_prefill_attngate_b200.HostPrefill): per KV-head
     # group, H2D of its Q/K/V, gate -> TopK mask -> sparse attention, D2H of its O, on three streams
     # so that the PCIe copies overlap the kernels.
-    hp = seer.HostPrefill(w.B, w.Hq, w.Hkv, w.S, w.d, w.d_gate, device=dev)
+    e2e_ms = e2e_value = None
+    if not args.no_e2e:
+        hp = seer.HostPrefill(w.B, w.Hq, w.Hkv, w.S, w.d, w.d_gate, device=dev)
 
-    def e2e_step():
-        hp.run(hq, hk, hv, hwq, hwk, ho, density=args.density, rope_theta=w.rope_theta)
+        def e2e_step():
+            hp.run(hq, hk, hv, hwq, hwk, ho, density=args.density, rope_theta=w.rope_theta)
 
-    for _ in range(2):
-        e2e_step()
-    torch.cuda.synchronize()
-    barrier(world)
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(e2e_steps):
-        e2e_step()
-    e1.record(stream)
-    torch.cuda.synchronize()
-    barrier(world)
-    seer.seer_check_status()
-    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps, world)
-    e2e_value = world * flops / (e2e_ms * 1e-3) / 1e12
+        for _ in range(2):
+            e2e_step()
+        torch.cuda.synchronize()
+        barrier(world)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(e2e_steps):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        barrier(world)
+        seer.seer_check_status()
+        e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps, world)
+        e2e_value = world * flops / (e2e_ms * 1e-3) / 1e12
 
     # ---------------- CPU baseline: the oracle on a bounded sample (rank 0, N=1)
     cpu_baseline = None
@@ -402,7 +404,7 @@ def run_gpu(args, world, rank, local):
                      "kernel": "attn_kernel<128,false> (seer_block_sparse_prefill)",
                      "algorithmic_flops_per_launch": flops},
         "density_sweep": sweep, "pooled_map": pooled, "decode": decode,
-        "e2e": {"value": round(e2e_value, 2), "unit": UNIT, "h2d_bytes_per_step": h2d,
+        "e2e": None if e2e_value is None else {"value": round(e2e_value, 2), "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 3)},
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clocks, "cpu_baseline": cpu_baseline, "wall_s_timed_region": round(t_wall, 3),
@@ -503,6 +505,7 @@ def main():
     ap.add_argument("--no-sweep", action="store_true")
     ap.add_argument("--no-map", action="store_true")
     ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true", help="skip the host-memory leg (profiling runs only)")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--ref-units", type=int, default=16)
