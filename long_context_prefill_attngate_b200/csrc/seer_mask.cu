@@ -199,7 +199,8 @@ __device__ __forceinline__ int row_k(int i, double density, int k_fixed, const i
 
 // One warp per row (rows of up to 32 * PER candidates): lane L holds the keys
 // of blocks j = 32 e + L.  The k-th largest key is found bit by bit from the
-// top (32 counting rounds, one warp reduction each); keys above it are kept,
+// top (up to 32 counting rounds, one warp reduction each, stopping as soon as
+// exactly k keys are at or above the prefix); keys above it are kept,
 // and among keys equal to it the lowest block indices, ranked with ballots.
 // Absent entries (j > i) hold key 0, below every real key.
 template <int PER>
@@ -242,6 +243,10 @@ __global__ void __launch_bounds__(256)
         cnt = __reduce_add_sync(0xffffffffu, cnt);
         if (cnt >= (unsigned)k)
             kth = cand;
+        // Exactly k keys at or above the prefix: they are the selection, and the
+        // lower bits cannot change it (the tie step below then takes all of them).
+        if (cnt == (unsigned)k)
+            break;
     }
     unsigned gt = 0;
 #pragma unroll
