@@ -326,6 +326,26 @@ def run_gpu(args, world, rank, local):
             tm.append(ev[1].elapsed_time(ev[2]))
             ta.append(ev[2].elapsed_time(ev[3]))
         seer.seer_check_status()
+        # steady state of a decoder: key rows cached, only the last (partial) block's row refreshed
+        kt = seer.seer_gate_key_cache(k, wk, rope_theta=w.rope_theta)
+        cws = torch.empty(seer.seer_workspace_bytes(seer.SEER_CALL_DECODE_GATE_CACHED, sh), dtype=torch.uint8,
+                          device=dev)
+        kws = torch.empty(seer.seer_workspace_bytes(seer.SEER_CALL_GATE_KEY_CACHE, sh), dtype=torch.uint8,
+                          device=dev)
+        tstep = []
+        for _ in range(10):
+            flush.zero_()
+            ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+            ev[0].record(stream)
+            seer.seer_gate_key_cache(k, wk, kt=kt, first_block=nb - 1, rope_theta=w.rope_theta, workspace=kws)
+            seer.seer_decode_gate_scores_cached(q_tok, kt, wq, w.S, w.Hkv, rope_theta=w.rope_theta, scores=ds,
+                                               workspace=cws)
+            seer.seer_decode_block_mask(ds, "topk", density=args.density, mask=dm)
+            seer.seer_block_sparse_decode(q_tok, k, v, dm, o=do, workspace=aws)
+            ev[1].record(stream)
+            torch.cuda.synchronize()
+            tstep.append(ev[0].elapsed_time(ev[1]))
+        seer.seer_check_status()
         g = w.Hq // w.Hkv
         union = int(dm.view(w.B, w.Hkv, g, nb).amax(2).sum().item())      # (KV head, block) pairs read
         kv_bytes = union * 64 * w.d * 2 * 2
@@ -333,9 +353,10 @@ def run_gpu(args, world, rank, local):
         decode = {"cache_tokens": w.S, "batch": w.B, "density": round(float(dm.float().mean().item()), 4),
                   "gate_us": round(statistics.median(tg) * 1e3, 1), "mask_us": round(statistics.median(tm) * 1e3, 1),
                   "attention_us": round(ms_a * 1e3, 1), "kv_bytes": kv_bytes,
+                  "step_us_cached_keys": round(statistics.median(tstep) * 1e3, 1),
                   "attention_gbs": round(kv_bytes / (ms_a * 1e-3) / 1e9, 1),
                   "frac_of_hbm_peak": round(kv_bytes / (ms_a * 1e-3) / 1e9 / pk["hbm_gbs"], 4)}
-        del dws, aws
+        del dws, aws, cws, kws, kt
 
     # ---------------- e2e: pinned host inputs -> C ABI -> host output, per step
     hq, hk, hv = (x[n].pin_memory() for n in ("q", "k", "v"))

@@ -110,7 +110,9 @@ enum {
     SEER_CALL_BLOCK_SPARSE_PREFILL = 1,
     SEER_CALL_ATTN_POOLED_MAP = 2,
     SEER_CALL_DECODE_GATE_SCORES = 3,
-    SEER_CALL_BLOCK_SPARSE_DECODE = 4
+    SEER_CALL_BLOCK_SPARSE_DECODE = 4,
+    SEER_CALL_GATE_KEY_CACHE = 5,
+    SEER_CALL_DECODE_GATE_CACHED = 6
 };
 
 /*
@@ -243,6 +245,31 @@ SEER_API seer_status seer_distill_loss(const seer_shape *shape, const float *sco
 SEER_API seer_status seer_decode_gate_scores(const seer_shape *shape, const void *q_tok, const void *k,
                                              const void *wq, const void *wk, const seer_gate_params *gp,
                                              float *scores, void *workspace, size_t ws_bytes, void *stream);
+
+/*
+ * seer_gate_key_cache — the gate's key rows Kt_j = RoPE_j(Kp_j @ Wk[h_kv])
+ * for blocks j = first_block .. nb-1 of a cache of shape->S = L tokens (the K
+ * side of seer_gate_scores and seer_decode_gate_scores).  A key row only
+ * changes while its block fills, so a decoder keeps kt across steps and
+ * refreshes from the last (partial) block on.  k: bf16 [B,Hkv,L,d]; wk and
+ * params as in seer_gate_scores; kt: fp32 [B,Hkv,nb,d_gate], rows below
+ * first_block untouched.  Workspace: seer_workspace_bytes(SEER_CALL_GATE_KEY_CACHE),
+ * 256-B aligned.
+ */
+SEER_API seer_status seer_gate_key_cache(const seer_shape *shape, const void *k, const void *wk,
+                                         const seer_gate_params *gp, int first_block, float *kt, void *workspace,
+                                         size_t ws_bytes, void *stream);
+
+/*
+ * seer_decode_gate_scores_cached — seer_decode_gate_scores on cached key
+ * rows: the token's q projected and rotated at block nb-1, softmax against
+ * kt (fp32 [B,Hkv,nb,d_gate], from seer_gate_key_cache).  scores: fp32
+ * [B,Hq,nb].  Workspace: seer_workspace_bytes(SEER_CALL_DECODE_GATE_CACHED),
+ * 256-B aligned.
+ */
+SEER_API seer_status seer_decode_gate_scores_cached(const seer_shape *shape, const void *q_tok, const float *kt,
+                                                    const void *wq, const seer_gate_params *gp, float *scores,
+                                                    void *workspace, size_t ws_bytes, void *stream);
 
 /*
  * seer_decode_block_mask — the mask row of the token: seer_block_mask's row

@@ -32,6 +32,8 @@ SEER_CALL_BLOCK_SPARSE_PREFILL = 1
 SEER_CALL_ATTN_POOLED_MAP = 2
 SEER_CALL_DECODE_GATE_SCORES = 3
 SEER_CALL_BLOCK_SPARSE_DECODE = 4
+SEER_CALL_GATE_KEY_CACHE = 5
+SEER_CALL_DECODE_GATE_CACHED = 6
 
 BLOCK = 64
 
@@ -41,6 +43,7 @@ EXPORTS = (
     "seer_attn_pooled_map", "seer_workspace_bytes", "seer_check_status", "seer_set_wait_timeout_ns",
     "seer_last_error", "seer_version", "seer_gate_scores_noalloc", "seer_distill_loss",
     "seer_decode_gate_scores", "seer_decode_block_mask", "seer_block_sparse_decode",
+    "seer_gate_key_cache", "seer_decode_gate_scores_cached",
 )
 
 
@@ -96,10 +99,12 @@ def lib() -> ctypes.CDLL:
             L.seer_decode_gate_scores.argtypes = [SP, P, P, P, P, ctypes.POINTER(seer_gate_params), P, P, Z, P]
             L.seer_decode_block_mask.argtypes = [SP, P, ctypes.POINTER(seer_mask_params), P, P]
             L.seer_block_sparse_decode.argtypes = [SP, P, P, P, P, F, P, P, P, Z, P]
+            L.seer_gate_key_cache.argtypes = [SP, P, P, ctypes.POINTER(seer_gate_params), I, P, P, Z, P]
+            L.seer_decode_gate_scores_cached.argtypes = [SP, P, P, P, ctypes.POINTER(seer_gate_params), P, P, Z, P]
             for fn in ("seer_gate_scores", "seer_gate_scores_noalloc", "seer_block_mask", "seer_compact_mask",
                        "seer_block_sparse_prefill", "seer_attn_pooled_map", "seer_check_status",
                        "seer_distill_loss", "seer_decode_gate_scores", "seer_decode_block_mask",
-                       "seer_block_sparse_decode"):
+                       "seer_block_sparse_decode", "seer_gate_key_cache", "seer_decode_gate_scores_cached"):
                 getattr(L, fn).restype = I
             L.seer_workspace_bytes.argtypes = [I, SP]
             L.seer_workspace_bytes.restype = Z
@@ -339,6 +344,49 @@ def seer_decode_gate_scores(q_tok, k, wq, wk, rope_theta: float = 5e5, scores=No
     gp = seer_gate_params(int(dg), float(rope_theta), int(wq_head_stride), int(wk_head_stride), int(bool(k_maxmin)))
     _check(lib().seer_decode_gate_scores(ctypes.byref(sh), _ptr(q_tok), _ptr(k), _ptr(wq), _ptr(wk),
                                          ctypes.byref(gp), _ptr(scores), _ptr(workspace), wsb, _stream_ptr(stream)))
+    return scores
+
+
+def seer_gate_key_cache(k, wk, kt=None, first_block: int = 0, rope_theta: float = 5e5, d_gate: int | None = None,
+                        workspace=None, stream=None, wk_head_stride: int | None = None, k_maxmin: bool = False):
+    """The gate's key rows fp32 [B,Hkv,nb,d_gate] for blocks first_block.. of the cache k [B,Hkv,L,d]
+    (rows below first_block of a given kt are left as they are)."""
+    torch = _torch()
+    _need(k.is_contiguous() and wk.is_contiguous() and k.dtype == wk.dtype == torch.bfloat16, "bf16 contiguous k, wk")
+    Bsz, Hkv, L, d = k.shape
+    dg = wk.shape[-1] if d_gate is None else d_gate
+    nb = -(-L // BLOCK)
+    sh = seer_shape(Bsz, Hkv, Hkv, L, d)
+    if wk_head_stride is None:
+        wk_head_stride = 0 if wk.dim() == 2 else (2 * d if k_maxmin else d) * dg
+    if kt is None:
+        kt = torch.empty((Bsz, Hkv, nb, dg), dtype=torch.float32, device=k.device)
+    _need(kt.dtype == torch.float32 and kt.is_contiguous() and tuple(kt.shape) == (Bsz, Hkv, nb, dg), "kt shape")
+    workspace, wsb = _workspace(SEER_CALL_GATE_KEY_CACHE, sh, k.device, workspace)
+    gp = seer_gate_params(int(dg), float(rope_theta), 0, int(wk_head_stride), int(bool(k_maxmin)))
+    _check(lib().seer_gate_key_cache(ctypes.byref(sh), _ptr(k), _ptr(wk), ctypes.byref(gp), int(first_block), _ptr(kt),
+                                     _ptr(workspace), wsb, _stream_ptr(stream)))
+    return kt
+
+
+def seer_decode_gate_scores_cached(q_tok, kt, wq, L: int, Hkv: int, rope_theta: float = 5e5, scores=None,
+                                   workspace=None, stream=None, wq_head_stride: int | None = None):
+    """Decode gate row fp32 [B,Hq,nb] from cached key rows kt [B,Hkv,nb,d_gate] (cache of L tokens)."""
+    torch = _torch()
+    _need(q_tok.is_contiguous() and wq.is_contiguous() and kt.is_contiguous(), "tensors must be contiguous")
+    Bsz, Hq, d = q_tok.shape
+    dg = wq.shape[-1]
+    nb = -(-L // BLOCK)
+    _need(tuple(kt.shape) == (Bsz, Hkv, nb, dg) and kt.dtype == torch.float32, "kt must be fp32 [B,Hkv,nb,d_gate]")
+    sh = seer_shape(Bsz, Hq, Hkv, L, d)
+    if wq_head_stride is None:
+        wq_head_stride = 0 if wq.dim() == 2 else d * dg
+    if scores is None:
+        scores = torch.empty((Bsz, Hq, nb), dtype=torch.float32, device=q_tok.device)
+    workspace, wsb = _workspace(SEER_CALL_DECODE_GATE_CACHED, sh, q_tok.device, workspace)
+    gp = seer_gate_params(int(dg), float(rope_theta), int(wq_head_stride), 0, 0)
+    _check(lib().seer_decode_gate_scores_cached(ctypes.byref(sh), _ptr(q_tok), _ptr(kt), _ptr(wq), ctypes.byref(gp),
+                                                _ptr(scores), _ptr(workspace), wsb, _stream_ptr(stream)))
     return scores
 
 

@@ -173,7 +173,12 @@ size_t seer_workspace_bytes(int which_call, const seer_shape *shape)
     case SEER_CALL_ATTN_POOLED_MAP:
         return sizeof(float) * (size_t)kMaxAttnCtas * nb * 128;
     case SEER_CALL_DECODE_GATE_SCORES:
-        return gate_workspace_bytes(shape->B, shape->Hq, shape->Hkv, shape->S, shape->d, 256, true);
+        return decode_gate_ws_bytes(shape->B, shape->Hq, shape->Hkv, shape->S, shape->d, 256, true);
+    case SEER_CALL_GATE_KEY_CACHE:
+        return gate_key_ws_bytes(shape->B, shape->Hkv, shape->S, shape->d, true);
+    case SEER_CALL_DECODE_GATE_CACHED:
+        return ((sizeof(float) * (size_t)shape->B * shape->Hq * shape->d + 255) & ~size_t(255)) +
+               ((sizeof(float) * (size_t)shape->B * shape->Hq * 256 + 255) & ~size_t(255));
     case SEER_CALL_BLOCK_SPARSE_DECODE:
         return sizeof(float) * (size_t)shape->B * shape->Hq * kMaxDecodeSplits * (shape->d + 2);
     default:
@@ -183,9 +188,11 @@ size_t seer_workspace_bytes(int which_call, const seer_shape *shape)
 }
 
 // Argument checks shared by the prefill and decode gates.
+// need_kind: 0 = the prefill gate's workspace, 1 = the decode gate's, 2 = the
+// key-cache call's, 3 = the cached decode row's.
 static seer_status check_gate_args(const char *name, const seer_shape *shape, const void *q, const void *k,
                                    const void *wq, const void *wk, const seer_gate_params *gp, const float *scores,
-                                   void *workspace, size_t ws_bytes)
+                                   void *workspace, size_t ws_bytes, int need_kind = 0)
 {
     seer_status st = check_shape(shape);
     if (st != SEER_OK)
@@ -208,8 +215,14 @@ static seer_status check_gate_args(const char *name, const seer_shape *shape, co
     if (gate_projection_smem(maxmin ? 2 * shape->d : shape->d, gp->d_gate) > 227 * 1024)
         return fail(SEER_ERR_UNSUPPORTED, "d_gate %d too large for %s K pooling at d = %d", gp->d_gate,
                     maxmin ? "max+min" : "average", shape->d);
-    const size_t need =
-        gate_workspace_bytes(shape->B, shape->Hq, shape->Hkv, shape->S, shape->d, gp->d_gate, maxmin);
+    size_t need = gate_workspace_bytes(shape->B, shape->Hq, shape->Hkv, shape->S, shape->d, gp->d_gate, maxmin);
+    if (need_kind == 1)
+        need = decode_gate_ws_bytes(shape->B, shape->Hq, shape->Hkv, shape->S, shape->d, gp->d_gate, maxmin);
+    else if (need_kind == 2)
+        need = gate_key_ws_bytes(shape->B, shape->Hkv, shape->S, shape->d, maxmin);
+    else if (need_kind == 3)   // the token's q rows, fp32, before and after the projection
+        need = ((sizeof(float) * (size_t)shape->B * shape->Hq * shape->d + 255) & ~size_t(255)) +
+               ((sizeof(float) * (size_t)shape->B * shape->Hq * gp->d_gate + 255) & ~size_t(255));
     if (workspace == nullptr || ws_bytes < need)
         return fail(SEER_ERR_WORKSPACE, "%s needs %zu workspace bytes, got %zu", name, need, ws_bytes);
     if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
@@ -411,7 +424,7 @@ seer_status seer_decode_gate_scores(const seer_shape *shape, const void *q_tok, 
                                     size_t ws_bytes, void *stream)
 {
     const seer_status st =
-        check_gate_args("seer_decode_gate_scores", shape, q_tok, k, wq, wk, gp, scores, workspace, ws_bytes);
+        check_gate_args("seer_decode_gate_scores", shape, q_tok, k, wq, wk, gp, scores, workspace, ws_bytes, 1);
     if (st != SEER_OK)
         return st;
     if (num_blocks(shape->S) * sizeof(float) + 1024 > 227 * 1024)
@@ -422,6 +435,42 @@ seer_status seer_decode_gate_scores(const seer_shape *shape, const void *q_tok, 
                                              static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess)
         return cuda_fail(e, "seer_decode_gate_scores launch");
+    return ok();
+}
+
+seer_status seer_gate_key_cache(const seer_shape *shape, const void *k, const void *wk, const seer_gate_params *gp,
+                                int first_block, float *kt, void *workspace, size_t ws_bytes, void *stream)
+{
+    // the q and wq checks of the shared helper are satisfied with k and wk
+    const seer_status st =
+        check_gate_args("seer_gate_key_cache", shape, k, k, wk, wk, gp, kt, workspace, ws_bytes, 2);
+    if (st != SEER_OK)
+        return st;
+    if (first_block < 0 || first_block > num_blocks(shape->S))
+        return fail(SEER_ERR_INVALID_ARG, "first_block %d outside [0, %d]", first_block, num_blocks(shape->S));
+    const cudaError_t e = launch_gate_keys(shape->B, shape->Hkv, shape->S, shape->d, gp->d_gate, gp->rope_theta,
+                                           gp->k_pooling == SEER_KPOOL_MAXMIN, k, wk, gp->wk_head_stride, first_block,
+                                           kt, workspace, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess)
+        return cuda_fail(e, "seer_gate_key_cache launch");
+    return ok();
+}
+
+seer_status seer_decode_gate_scores_cached(const seer_shape *shape, const void *q_tok, const float *kt,
+                                           const void *wq, const seer_gate_params *gp, float *scores, void *workspace,
+                                           size_t ws_bytes, void *stream)
+{
+    const seer_status st = check_gate_args("seer_decode_gate_scores_cached", shape, q_tok, kt, wq, wq, gp, scores,
+                                           workspace, ws_bytes, 3);
+    if (st != SEER_OK)
+        return st;
+    if ((reinterpret_cast<uintptr_t>(kt) & 15u) != 0)
+        return fail(SEER_ERR_INVALID_ARG, "kt must be 16-byte aligned");
+    const cudaError_t e = launch_decode_gate_cached(shape->B, shape->Hq, shape->Hkv, shape->S, shape->d, gp->d_gate,
+                                                    gp->rope_theta, q_tok, wq, gp->wq_head_stride, kt, scores,
+                                                    workspace, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess)
+        return cuda_fail(e, "seer_decode_gate_scores_cached launch");
     return ok();
 }
 

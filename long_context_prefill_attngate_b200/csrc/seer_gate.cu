@@ -29,15 +29,16 @@ constexpr int kPoolThreads = 128;
 // (2D features per block) — the K pooling variant of the gate.
 template <int D, bool MAXMIN = false>
 __global__ void __launch_bounds__(kPoolThreads) pool_kernel(const __nv_bfloat16 *__restrict__ x, int S, int nb,
-                                                            float *__restrict__ out)
+                                                            int first, float *__restrict__ out)
 {
     constexpr int CH = D / 8;                 // 16-byte chunks per row
     constexpr int RPI = kPoolThreads / CH;    // rows handled in parallel
     __shared__ float part[RPI][D];
     __shared__ float part2[MAXMIN ? RPI : 1][MAXMIN ? D : 1];
-    const long long blk = blockIdx.x;         // = bh * nb + i
-    const long long bh = blk / nb;
-    const int i = (int)(blk % nb);
+    // blocks first .. nb-1 of every head: blockIdx.x = bh * (nb - first) + (i - first)
+    const long long bh = (long long)blockIdx.x / (nb - first);
+    const int i = first + (int)(blockIdx.x % (nb - first));
+    const long long blk = bh * nb + i;         // output row
     const int rows = min(64, S - 64 * i);      // tokens in this block
     const __nv_bfloat16 *base = x + (bh * S + 64LL * i) * D;
     const int c = threadIdx.x % CH;
@@ -104,14 +105,16 @@ constexpr int kPA = kProjRows / 16;         // rows per thread
 constexpr int kProjThreads = 256;      // 16 x 16: rows ty + 16a, rotation pairs tx + 16b
 constexpr int kPStride = 4;            // padding (floats) of the shared rows
 
-// out[bh, i, :] = RoPE_{pos0+i}( xp[bh, i, :] @ W[h] ) for kProjRows rows i of one
+// out[bh, i, :] = RoPE_{pos0+i}( xp[bh, i, :] @ W[h] ) for i < nb (rows ld apart
+// between heads), kProjRows rows i of one
 // head.  Each thread owns kPA rows x 4 rotation pairs (t, t + dg/2), so both halves
 // of a pair are in its registers when the rotation is applied.  Angles
 // i * theta^(-2t/dg): frequencies in double once per CTA, angle formed and
 // reduced modulo 2*pi in double, the reduced angle through fp32 sincosf.
 __global__ void __launch_bounds__(kProjThreads)
-    project_rope_kernel(const float *__restrict__ xp, int H, int nb, int d, const __nv_bfloat16 *__restrict__ w,
-                        long long w_stride, int dg, double theta, int pos0, float *__restrict__ out)
+    project_rope_kernel(const float *__restrict__ xp, int H, int nb, int ld, int d,
+                        const __nv_bfloat16 *__restrict__ w, long long w_stride, int dg, double theta, int pos0,
+                        float *__restrict__ out)
 {
     extern __shared__ float4 psm4[];
     const int xs = d + kPStride;
@@ -141,7 +144,7 @@ __global__ void __launch_bounds__(kProjThreads)
         for (int e = threadIdx.x; e < d * dg; e += kProjThreads)
             sw[e] = __bfloat162float(wh[e]);
     }
-    const float *xb = xp + ((long long)bh * nb + i0) * d;
+    const float *xb = xp + ((long long)bh * ld + i0) * d;
     for (int e = threadIdx.x; e < kProjRows * d; e += kProjThreads) {
         const int r = e / d, c = e % d;
         sx[r * xs + c] = r < rows ? xb[e] : 0.f;
@@ -187,7 +190,7 @@ __global__ void __launch_bounds__(kProjThreads)
             if (r >= rows)
                 continue;
             const int i = i0 + r;
-            float *o = out + ((long long)bh * nb + i) * dg;
+            float *o = out + ((long long)bh * ld + i) * dg;
 #pragma unroll
             for (int b = 0; b < 4; ++b) {
                 const int t = t0 + tx + 16 * b;
@@ -448,17 +451,17 @@ cudaError_t launch_gate(int B, int Hq, int Hkv, int S, int d, int dg, float thet
     const auto *kb = static_cast<const __nv_bfloat16 *>(k);
     const unsigned gq = (unsigned)((long long)B * Hq * nb), gk = (unsigned)((long long)B * Hkv * nb);
     if (d == 128) {
-        pool_kernel<128><<<gq, kPoolThreads, 0, stream>>>(qb, S, nb, qp);
+        pool_kernel<128><<<gq, kPoolThreads, 0, stream>>>(qb, S, nb, 0, qp);
         if (k_maxmin)
-            pool_kernel<128, true><<<gk, kPoolThreads, 0, stream>>>(kb, S, nb, kp);
+            pool_kernel<128, true><<<gk, kPoolThreads, 0, stream>>>(kb, S, nb, 0, kp);
         else
-            pool_kernel<128><<<gk, kPoolThreads, 0, stream>>>(kb, S, nb, kp);
+            pool_kernel<128><<<gk, kPoolThreads, 0, stream>>>(kb, S, nb, 0, kp);
     } else {
-        pool_kernel<64><<<gq, kPoolThreads, 0, stream>>>(qb, S, nb, qp);
+        pool_kernel<64><<<gq, kPoolThreads, 0, stream>>>(qb, S, nb, 0, qp);
         if (k_maxmin)
-            pool_kernel<64, true><<<gk, kPoolThreads, 0, stream>>>(kb, S, nb, kp);
+            pool_kernel<64, true><<<gk, kPoolThreads, 0, stream>>>(kb, S, nb, 0, kp);
         else
-            pool_kernel<64><<<gk, kPoolThreads, 0, stream>>>(kb, S, nb, kp);
+            pool_kernel<64><<<gk, kPoolThreads, 0, stream>>>(kb, S, nb, 0, kp);
     }
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess)
@@ -470,10 +473,10 @@ cudaError_t launch_gate(int B, int Hq, int Hkv, int S, int d, int dg, float thet
     const size_t psmem_q = gate_projection_smem(d, dg);
     const dim3 pg_q((nb + kProjRows - 1) / kProjRows, B * Hq);
     const dim3 pg_k((nb + kProjRows - 1) / kProjRows, B * Hkv);
-    project_rope_kernel<<<pg_q, kProjThreads, psmem_q, stream>>>(qp, Hq, nb, d,
+    project_rope_kernel<<<pg_q, kProjThreads, psmem_q, stream>>>(qp, Hq, nb, nb, d,
                                                                static_cast<const __nv_bfloat16 *>(wq), wq_stride,
                                                                dg, (double)theta, 0, qt);
-    project_rope_kernel<<<pg_k, kProjThreads, psmem, stream>>>(kp, Hkv, nb, dk,
+    project_rope_kernel<<<pg_k, kProjThreads, psmem, stream>>>(kp, Hkv, nb, nb, dk,
                                                                static_cast<const __nv_bfloat16 *>(wk), wk_stride,
                                                                dg, (double)theta, 0, kt);
     e = cudaGetLastError();
@@ -492,41 +495,35 @@ cudaError_t launch_gate(int B, int Hq, int Hkv, int S, int d, int dg, float thet
 
 namespace seer {
 
-// Decode gate ("SeerAttention-R": the gate without query pooling): the K side
-// is the prefill gate's (pooled K of the L-token cache, projected, block
-// RoPE); the token's q is projected and rotated at its block, nb - 1.  The
-// workspace layout is the prefill gate's (its Q regions hold the q rows).
-cudaError_t launch_decode_gate(int B, int Hq, int Hkv, int L, int d, int dg, float theta, bool k_maxmin,
-                               const void *q_tok, const void *k, const void *wq, long long wq_stride, const void *wk,
-                               long long wk_stride, float *scores, void *ws, cudaStream_t stream)
+// Decode gate ("SeerAttention-R": the gate without query pooling).  Its K
+// side is the prefill gate's: pooled K of the L-token cache, projected, block
+// RoPE, one row per block.  Those rows only change when a block changes, so
+// they are exposed as a cache: launch_gate_keys (re)computes rows
+// first_block .. nb-1, and launch_decode_gate_cached projects the token's q at
+// block nb - 1 and takes the row softmax against the cached rows.
+cudaError_t launch_gate_keys(int B, int Hkv, int L, int d, int dg, float theta, bool k_maxmin, const void *k,
+                             const void *wk, long long wk_stride, int first_block, float *kt, void *ws,
+                             cudaStream_t stream)
 {
     const int nb = num_blocks(L);
     const int dk = k_maxmin ? 2 * d : d;
-    char *p = static_cast<char *>(ws);
-    float *qp = reinterpret_cast<float *>(p);
-    p += align256(sizeof(float) * B * Hq * (size_t)nb * d);
-    float *kp = reinterpret_cast<float *>(p);
-    p += align256(sizeof(float) * B * Hkv * (size_t)nb * dk);
-    float *qt = reinterpret_cast<float *>(p);
-    p += align256(sizeof(float) * B * Hq * (size_t)nb * dg);
-    float *kt = reinterpret_cast<float *>(p);
-
+    const int nsel = nb - first_block;
+    if (nsel <= 0)
+        return cudaSuccess;
+    float *kp = static_cast<float *>(ws);                    // [B*Hkv, nb, dk]; rows >= first_block written
     const auto *kb = static_cast<const __nv_bfloat16 *>(k);
-    const unsigned gk = (unsigned)((long long)B * Hkv * nb);
+    const unsigned gk = (unsigned)((long long)B * Hkv * nsel);
     if (d == 128) {
         if (k_maxmin)
-            pool_kernel<128, true><<<gk, kPoolThreads, 0, stream>>>(kb, L, nb, kp);
+            pool_kernel<128, true><<<gk, kPoolThreads, 0, stream>>>(kb, L, nb, first_block, kp);
         else
-            pool_kernel<128><<<gk, kPoolThreads, 0, stream>>>(kb, L, nb, kp);
+            pool_kernel<128><<<gk, kPoolThreads, 0, stream>>>(kb, L, nb, first_block, kp);
     } else {
         if (k_maxmin)
-            pool_kernel<64, true><<<gk, kPoolThreads, 0, stream>>>(kb, L, nb, kp);
+            pool_kernel<64, true><<<gk, kPoolThreads, 0, stream>>>(kb, L, nb, first_block, kp);
         else
-            pool_kernel<64><<<gk, kPoolThreads, 0, stream>>>(kb, L, nb, kp);
+            pool_kernel<64><<<gk, kPoolThreads, 0, stream>>>(kb, L, nb, first_block, kp);
     }
-    const long long nq = (long long)B * Hq * d;
-    q_to_f32_kernel<<<(unsigned)((nq + 255) / 256), 256, 0, stream>>>(static_cast<const __nv_bfloat16 *>(q_tok), nq,
-                                                                       qp);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess)
         return e;
@@ -534,11 +531,30 @@ cudaError_t launch_decode_gate(int B, int Hq, int Hkv, int L, int d, int dg, flo
     e = cudaFuncSetAttribute(project_rope_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)psmem);
     if (e != cudaSuccess)
         return e;
-    // q: one row per head at position nb - 1; K: every block.
-    project_rope_kernel<<<dim3(1, B * Hq), kProjThreads, gate_projection_smem(d, dg), stream>>>(
-        qp, Hq, 1, d, static_cast<const __nv_bfloat16 *>(wq), wq_stride, dg, (double)theta, nb - 1, qt);
-    project_rope_kernel<<<dim3((nb + kProjRows - 1) / kProjRows, B * Hkv), kProjThreads, psmem, stream>>>(
-        kp, Hkv, nb, dk, static_cast<const __nv_bfloat16 *>(wk), wk_stride, dg, (double)theta, 0, kt);
+    project_rope_kernel<<<dim3((nsel + kProjRows - 1) / kProjRows, B * Hkv), kProjThreads, psmem, stream>>>(
+        kp + (size_t)first_block * dk, Hkv, nsel, nb, dk, static_cast<const __nv_bfloat16 *>(wk), wk_stride, dg,
+        (double)theta, first_block, kt + (size_t)first_block * dg);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_decode_gate_cached(int B, int Hq, int Hkv, int L, int d, int dg, float theta, const void *q_tok,
+                                      const void *wq, long long wq_stride, const float *kt, float *scores, void *ws,
+                                      cudaStream_t stream)
+{
+    const int nb = num_blocks(L);
+    float *qp = static_cast<float *>(ws);                               // [B*Hq, d]
+    float *qt = qp + align256(sizeof(float) * (size_t)B * Hq * d) / sizeof(float);   // [B*Hq, dg]
+    const long long nq = (long long)B * Hq * d;
+    q_to_f32_kernel<<<(unsigned)((nq + 255) / 256), 256, 0, stream>>>(static_cast<const __nv_bfloat16 *>(q_tok), nq,
+                                                                       qp);
+    const size_t psmem_q = gate_projection_smem(d, dg);
+    cudaError_t e = cudaFuncSetAttribute(project_rope_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)gate_projection_smem(2 * d, dg));
+    if (e != cudaSuccess)
+        return e;
+    // the token's q: one row per head, rotated at its block, nb - 1
+    project_rope_kernel<<<dim3(1, B * Hq), kProjThreads, psmem_q, stream>>>(
+        qp, Hq, 1, 1, d, static_cast<const __nv_bfloat16 *>(wq), wq_stride, dg, (double)theta, nb - 1, qt);
     e = cudaGetLastError();
     if (e != cudaSuccess)
         return e;
@@ -549,6 +565,33 @@ cudaError_t launch_decode_gate(int B, int Hq, int Hkv, int L, int d, int dg, flo
     decode_gate_kernel<<<B * Hq, kDecThreads, dsmem, stream>>>(qt, kt, Hq, Hkv, nb, dg, 1.0f / sqrtf((float)dg),
                                                                 scores);
     return cudaGetLastError();
+}
+
+size_t gate_key_ws_bytes(int B, int Hkv, int L, int d, bool k_maxmin)
+{
+    return align256(sizeof(float) * (size_t)B * Hkv * num_blocks(L) * (k_maxmin ? 2 * d : d));
+}
+
+size_t decode_gate_ws_bytes(int B, int Hq, int Hkv, int L, int d, int dg, bool k_maxmin)
+{
+    // the cached-row part, then the key rows and the key-pooling scratch
+    const size_t q = align256(sizeof(float) * (size_t)B * Hq * d) + align256(sizeof(float) * (size_t)B * Hq * dg);
+    return q + align256(sizeof(float) * (size_t)B * Hkv * num_blocks(L) * dg) + gate_key_ws_bytes(B, Hkv, L, d, k_maxmin);
+}
+
+// The whole decode gate: key rows for every block, then the token's row.
+cudaError_t launch_decode_gate(int B, int Hq, int Hkv, int L, int d, int dg, float theta, bool k_maxmin,
+                               const void *q_tok, const void *k, const void *wq, long long wq_stride, const void *wk,
+                               long long wk_stride, float *scores, void *ws, cudaStream_t stream)
+{
+    char *p = static_cast<char *>(ws);
+    const size_t q = align256(sizeof(float) * (size_t)B * Hq * d) + align256(sizeof(float) * (size_t)B * Hq * dg);
+    float *kt = reinterpret_cast<float *>(p + q);
+    void *kws = p + q + align256(sizeof(float) * (size_t)B * Hkv * num_blocks(L) * dg);
+    cudaError_t e = launch_gate_keys(B, Hkv, L, d, dg, theta, k_maxmin, k, wk, wk_stride, 0, kt, kws, stream);
+    if (e != cudaSuccess)
+        return e;
+    return launch_decode_gate_cached(B, Hq, Hkv, L, d, dg, theta, q_tok, wq, wq_stride, kt, scores, ws, stream);
 }
 
 } // namespace seer

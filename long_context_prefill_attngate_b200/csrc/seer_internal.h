@@ -46,6 +46,14 @@ size_t gate_projection_smem(int d_in, int dg);
 cudaError_t launch_decode_gate(int B, int Hq, int Hkv, int L, int d, int dg, float theta, bool k_maxmin,
                                const void *q_tok, const void *k, const void *wq, long long wq_stride, const void *wk,
                                long long wk_stride, float *scores, void *ws, cudaStream_t stream);
+cudaError_t launch_gate_keys(int B, int Hkv, int L, int d, int dg, float theta, bool k_maxmin, const void *k,
+                             const void *wk, long long wk_stride, int first_block, float *kt, void *ws,
+                             cudaStream_t stream);
+cudaError_t launch_decode_gate_cached(int B, int Hq, int Hkv, int L, int d, int dg, float theta, const void *q_tok,
+                                      const void *wq, long long wq_stride, const float *kt, float *scores, void *ws,
+                                      cudaStream_t stream);
+size_t gate_key_ws_bytes(int B, int Hkv, int L, int d, bool k_maxmin);
+size_t decode_gate_ws_bytes(int B, int Hq, int Hkv, int L, int d, int dg, bool k_maxmin);
 
 // Block-sparse decode attention (seer_decode.cu).
 constexpr int kMaxDecodeSplits = 64;

@@ -144,3 +144,34 @@ def test_decode_step_full_size(oracle):
     o_ref, lse_ref = oracle.decode_attention(bits(q), bits(k), bits(v), m.cpu().numpy())
     check_o(o, o_ref, "decode O (32k)")
     assert np.abs(lse.cpu().double().numpy() - lse_ref).max() <= 1e-3
+
+
+@pytest.mark.parametrize("maxmin", [False, True])
+def test_decode_gate_key_cache(oracle, maxmin):
+    """Key rows kept across decode steps: the cached row equals the one-call
+    gate bit for bit, and refreshing only from the last partial block on after
+    the cache grew equals recomputing every row."""
+    B, Hq, Hkv, d, dg = 2, 8, 2, 128, 64
+    L1, L2 = 5 * BLOCK + 10, 6 * BLOCK + 3
+    w, q, k, v, wq, wk = decode_inputs(B, Hq, Hkv, L2, d, dg, 361)
+    if maxmin:
+        g = torch.Generator().manual_seed(361)
+        wk = (torch.randn((Hkv, 2 * d, dg), generator=g) * 0.08).to(torch.bfloat16)
+    kd, wqd, wkd, qd = dev(k), dev(wq), dev(wk), dev(q)
+    k1 = kd[:, :, :L1].contiguous()
+    kt1 = seer.seer_gate_key_cache(k1, wkd, rope_theta=w.rope_theta, k_maxmin=maxmin)
+    s_c = seer.seer_decode_gate_scores_cached(qd, kt1, wqd, L1, Hkv, rope_theta=w.rope_theta)
+    s_f = seer.seer_decode_gate_scores(qd, k1, wqd, wkd, rope_theta=w.rope_theta, k_maxmin=maxmin)
+    seer.seer_check_status()
+    assert torch.equal(s_c, s_f)
+    ref = oracle.decode_gate_scores(bits(q), bits(k[:, :, :L1]), bits(wq), bits(wk), theta=w.rope_theta,
+                                    k_maxmin=maxmin)
+    check_rel(s_c.cpu().numpy(), ref, "cached decode scores")
+    # the cache grows to L2: keep the complete blocks, refresh from block 5 (was partial) on
+    nb1, nb2 = -(-L1 // BLOCK), -(-L2 // BLOCK)
+    kt2 = torch.full((B, Hkv, nb2, dg), float("nan"), dtype=torch.float32, device="cuda")
+    kt2[:, :, : nb1 - 1] = kt1[:, :, : nb1 - 1]
+    seer.seer_gate_key_cache(kd, wkd, kt=kt2, first_block=nb1 - 1, rope_theta=w.rope_theta, k_maxmin=maxmin)
+    full = seer.seer_gate_key_cache(kd, wkd, rope_theta=w.rope_theta, k_maxmin=maxmin)
+    seer.seer_check_status()
+    assert torch.equal(kt2, full)
