@@ -27,17 +27,17 @@ constexpr int kPoolThreads = 128;
 // bf16 values (64, or the S - 64 i tokens of a ragged last block).
 // MAXMIN: per-block max and min instead of the mean, written [max | min]
 // (2D features per block) — the K pooling variant of the gate.
-template <int D, bool MAXMIN = false>
-__global__ void __launch_bounds__(kPoolThreads) pool_kernel(const __nv_bfloat16 *__restrict__ x, int S, int nb,
-                                                            int first, float *__restrict__ out)
+template <int D, bool MAXMIN>
+__device__ __forceinline__ void pool_block(const __nv_bfloat16 *__restrict__ x, int S, int nb, int first,
+                                           float *__restrict__ out, unsigned cta)
 {
     constexpr int CH = D / 8;                 // 16-byte chunks per row
     constexpr int RPI = kPoolThreads / CH;    // rows handled in parallel
     __shared__ float part[RPI][D];
     __shared__ float part2[MAXMIN ? RPI : 1][MAXMIN ? D : 1];
-    // blocks first .. nb-1 of every head: blockIdx.x = bh * (nb - first) + (i - first)
-    const long long bh = (long long)blockIdx.x / (nb - first);
-    const int i = first + (int)(blockIdx.x % (nb - first));
+    // blocks first .. nb-1 of every head: cta = bh * (nb - first) + (i - first)
+    const long long bh = (long long)cta / (nb - first);
+    const int i = first + (int)(cta % (nb - first));
     const long long blk = bh * nb + i;         // output row
     const int rows = min(64, S - 64 * i);      // tokens in this block
     const __nv_bfloat16 *base = x + (bh * S + 64LL * i) * D;
@@ -100,6 +100,27 @@ __global__ void __launch_bounds__(kPoolThreads) pool_kernel(const __nv_bfloat16 
     }
 }
 
+template <int D, bool MAXMIN = false>
+__global__ void __launch_bounds__(kPoolThreads) pool_kernel(const __nv_bfloat16 *__restrict__ x, int S, int nb,
+                                                            int first, float *__restrict__ out)
+{
+    pool_block<D, MAXMIN>(x, S, nb, first, out, blockIdx.x);
+}
+
+// Mean pooling of Q and K in one launch: CTAs below nq pool Q, the rest K
+// (the two grids would otherwise run back to back, each with its own tail).
+template <int D>
+__global__ void __launch_bounds__(kPoolThreads) pool_qk_kernel(const __nv_bfloat16 *__restrict__ q,
+                                                               float *__restrict__ qp, unsigned nq,
+                                                               const __nv_bfloat16 *__restrict__ k,
+                                                               float *__restrict__ kp, int S, int nb)
+{
+    if (blockIdx.x < nq)
+        pool_block<D, false>(q, S, nb, 0, qp, blockIdx.x);
+    else
+        pool_block<D, false>(k, S, nb, 0, kp, blockIdx.x - nq);
+}
+
 constexpr int kProjRows = 64;               // query/key blocks per CTA (16 and 32 measured no faster)
 constexpr int kPA = kProjRows / 16;         // rows per thread
 constexpr int kProjThreads = 256;      // 16 x 16: rows ty + 16a, rotation pairs tx + 16b
@@ -111,17 +132,33 @@ constexpr int kPStride = 4;            // padding (floats) of the shared rows
 // of a pair are in its registers when the rotation is applied.  Angles
 // i * theta^(-2t/dg): frequencies in double once per CTA, angle formed and
 // reduced modulo 2*pi in double, the reduced angle through fp32 sincosf.
+struct ProjJob {
+    const float *xp;                 // pooled rows [B*H, ld, d]
+    int H, d;
+    const __nv_bfloat16 *w;          // [H] x (d x dg), w_stride apart
+    long long w_stride;
+    float *out;                      // [B*H, ld, dg]
+};
+
+// Two projections in one launch: grid rows blockIdx.y < ny0 run job j0, the
+// rest job j1 (the Q and K sides of the gate, which would otherwise leave
+// most of the GPU idle in the smaller launch).
 __global__ void __launch_bounds__(kProjThreads)
-    project_rope_kernel(const float *__restrict__ xp, int H, int nb, int ld, int d,
-                        const __nv_bfloat16 *__restrict__ w, long long w_stride, int dg, double theta, int pos0,
-                        float *__restrict__ out)
+    project_rope_kernel(ProjJob j0, ProjJob j1, int ny0, int nb, int ld, int dg, double theta, int pos0)
 {
     extern __shared__ float4 psm4[];
+    const bool second = (int)blockIdx.y >= ny0;
+    const ProjJob &job = second ? j1 : j0;
+    const float *__restrict__ xp = job.xp;
+    const int H = job.H, d = job.d;
+    const __nv_bfloat16 *__restrict__ w = job.w;
+    const long long w_stride = job.w_stride;
+    float *__restrict__ out = job.out;
     const int xs = d + kPStride;
     float *sx = reinterpret_cast<float *>(psm4);           // kProjRows x xs
     float *sw = sx + kProjRows * xs;                       // d x dg (fp32)
     double *sfreq = reinterpret_cast<double *>(sw + d * dg);
-    const int bh = blockIdx.y;
+    const int bh = (int)blockIdx.y - (second ? ny0 : 0);
     const int h = bh % H;
     const int i0 = blockIdx.x * kProjRows;
     const int rows = min(kProjRows, nb - i0);
@@ -208,9 +245,10 @@ __global__ void __launch_bounds__(kProjThreads)
 }
 
 constexpr int kLR = 32;              // query blocks per CTA (16, 64, 128 measured slower)
-constexpr int kLA = kLR / 16;        // query rows per thread
-constexpr int kLC = 64;              // key blocks per tile
 constexpr int kLThreads = 256;       // 16 x 16: rows ty + 16a, columns tx + 16b
+constexpr int kLTy = kLThreads / 16; // thread rows
+constexpr int kLA = kLR / kLTy;      // query rows per thread
+constexpr int kLC = 64;              // key blocks per tile
 constexpr int kLPad = 4;             // row padding (floats): conflict-free float4 reads
 
 // Causal block logits + row softmax for kLR query blocks of one head.  Each
@@ -219,6 +257,9 @@ constexpr int kLPad = 4;             // row padding (floats): conflict-free floa
 // each row's running max and exp-sum are kept online (the 16 threads sharing
 // a row reduce with shuffles).  A second pass over the same tiles writes
 // exp(x - m) / sum, and the entries j > i are set to 0.
+constexpr int kLPF = 8;              // float4 per thread of a prefetched Kt tile (d_gate <= 128)
+
+template <bool PF>
 __global__ void __launch_bounds__(kLThreads)
     gate_softmax_kernel(const float *__restrict__ qt, const float *__restrict__ kt, int Hq, int Hkv, int nb, int dg,
                         float scale, float *__restrict__ scores)
@@ -250,28 +291,54 @@ __global__ void __launch_bounds__(kLThreads)
         m[a] = -INFINITY;
         ssum[a] = 0.f;
     }
+    // PF: the next Kt tile is loaded into registers while this one is used,
+    // hiding the L2 latency of the tile loads.
+    float4 pf[PF ? kLPF : 1];
+    auto fetch = [&](int jt) {
+        const int nc = min(kLC, jlast + 1 - jt);
+#pragma unroll
+        for (int it = 0; it < kLPF; ++it) {
+            const int e = threadIdx.x + it * kLThreads;
+            const int jj = e / dg4, c4 = e % dg4;
+            pf[it] = (e < kLC * dg4 && jj < nc) ? reinterpret_cast<const float4 *>(kbase + (long long)(jt + jj) * dg)[c4]
+                                                : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+    };
+    if (PF)
+        fetch(0);
     for (int j0 = 0; j0 <= jlast; j0 += kLC) {
         __syncthreads();
-        const int ncols = min(kLC, jlast + 1 - j0);
-        for (int e = threadIdx.x; e < kLC * dg4; e += kLThreads) {
-            const int jj = e / dg4, c4 = e % dg4;
-            const float4 v = jj < ncols ? reinterpret_cast<const float4 *>(kbase + (long long)(j0 + jj) * dg)[c4]
-                                        : make_float4(0.f, 0.f, 0.f, 0.f);
-            *reinterpret_cast<float4 *>(sk + jj * rs + 4 * c4) = v;
+        if (PF) {
+#pragma unroll
+            for (int it = 0; it < kLPF; ++it) {
+                const int e = threadIdx.x + it * kLThreads;
+                if (e < kLC * dg4)
+                    *reinterpret_cast<float4 *>(sk + (e / dg4) * rs + 4 * (e % dg4)) = pf[it];
+            }
+        } else {
+            const int ncols = min(kLC, jlast + 1 - j0);
+            for (int e = threadIdx.x; e < kLC * dg4; e += kLThreads) {
+                const int jj = e / dg4, c4 = e % dg4;
+                const float4 v = jj < ncols ? reinterpret_cast<const float4 *>(kbase + (long long)(j0 + jj) * dg)[c4]
+                                            : make_float4(0.f, 0.f, 0.f, 0.f);
+                *reinterpret_cast<float4 *>(sk + jj * rs + 4 * c4) = v;
+            }
         }
         __syncthreads();
+        if (PF && j0 + kLC <= jlast)
+            fetch(j0 + kLC);
         float acc[kLA][4];
 #pragma unroll
         for (int a = 0; a < kLA; ++a)
 #pragma unroll
             for (int c = 0; c < 4; ++c)
                 acc[a][c] = 0.f;
-#pragma unroll 2
+#pragma unroll 1
         for (int c = 0; c < dg; c += 4) {
             float4 qv[kLA], kv[4];
 #pragma unroll
             for (int a = 0; a < kLA; ++a)
-                qv[a] = *reinterpret_cast<const float4 *>(sq + (ty + 16 * a) * rs + c);
+                qv[a] = *reinterpret_cast<const float4 *>(sq + (ty + kLTy * a) * rs + c);
 #pragma unroll
             for (int bb = 0; bb < 4; ++bb)
                 kv[bb] = *reinterpret_cast<const float4 *>(sk + (tx + 16 * bb) * rs + c);
@@ -284,7 +351,7 @@ __global__ void __launch_bounds__(kLThreads)
         }
 #pragma unroll
         for (int a = 0; a < kLA; ++a) {
-            const int r = ty + 16 * a;
+            const int r = ty + kLTy * a;
             const int i = i0 + r;
             float tm = -INFINITY;
 #pragma unroll
@@ -320,7 +387,7 @@ __global__ void __launch_bounds__(kLThreads)
     for (int j0 = 0; j0 <= jlast; j0 += kLC) {
 #pragma unroll
         for (int a = 0; a < kLA; ++a) {
-            const int r = ty + 16 * a;
+            const int r = ty + kLTy * a;
             const int i = i0 + r;
             if (r >= rows)
                 continue;
@@ -450,44 +517,45 @@ cudaError_t launch_gate(int B, int Hq, int Hkv, int S, int d, int dg, float thet
     const auto *qb = static_cast<const __nv_bfloat16 *>(q);
     const auto *kb = static_cast<const __nv_bfloat16 *>(k);
     const unsigned gq = (unsigned)((long long)B * Hq * nb), gk = (unsigned)((long long)B * Hkv * nb);
-    if (d == 128) {
-        pool_kernel<128><<<gq, kPoolThreads, 0, stream>>>(qb, S, nb, 0, qp);
-        if (k_maxmin)
-            pool_kernel<128, true><<<gk, kPoolThreads, 0, stream>>>(kb, S, nb, 0, kp);
+    if (!k_maxmin) {
+        if (d == 128)
+            pool_qk_kernel<128><<<gq + gk, kPoolThreads, 0, stream>>>(qb, qp, gq, kb, kp, S, nb);
         else
-            pool_kernel<128><<<gk, kPoolThreads, 0, stream>>>(kb, S, nb, 0, kp);
+            pool_qk_kernel<64><<<gq + gk, kPoolThreads, 0, stream>>>(qb, qp, gq, kb, kp, S, nb);
+    } else if (d == 128) {
+        pool_kernel<128><<<gq, kPoolThreads, 0, stream>>>(qb, S, nb, 0, qp);
+        pool_kernel<128, true><<<gk, kPoolThreads, 0, stream>>>(kb, S, nb, 0, kp);
     } else {
         pool_kernel<64><<<gq, kPoolThreads, 0, stream>>>(qb, S, nb, 0, qp);
-        if (k_maxmin)
-            pool_kernel<64, true><<<gk, kPoolThreads, 0, stream>>>(kb, S, nb, 0, kp);
-        else
-            pool_kernel<64><<<gk, kPoolThreads, 0, stream>>>(kb, S, nb, 0, kp);
+        pool_kernel<64, true><<<gk, kPoolThreads, 0, stream>>>(kb, S, nb, 0, kp);
     }
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess)
         return e;
-    const size_t psmem = gate_projection_smem(dk, dg);
+    const size_t psmem = gate_projection_smem(dk, dg);    // dk >= d: covers both jobs
     e = cudaFuncSetAttribute(project_rope_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)psmem);
     if (e != cudaSuccess)
         return e;
-    const size_t psmem_q = gate_projection_smem(d, dg);
-    const dim3 pg_q((nb + kProjRows - 1) / kProjRows, B * Hq);
-    const dim3 pg_k((nb + kProjRows - 1) / kProjRows, B * Hkv);
-    project_rope_kernel<<<pg_q, kProjThreads, psmem_q, stream>>>(qp, Hq, nb, nb, d,
-                                                               static_cast<const __nv_bfloat16 *>(wq), wq_stride,
-                                                               dg, (double)theta, 0, qt);
-    project_rope_kernel<<<pg_k, kProjThreads, psmem, stream>>>(kp, Hkv, nb, nb, dk,
-                                                               static_cast<const __nv_bfloat16 *>(wk), wk_stride,
-                                                               dg, (double)theta, 0, kt);
+    const ProjJob jq{qp, Hq, d, static_cast<const __nv_bfloat16 *>(wq), wq_stride, qt};
+    const ProjJob jk{kp, Hkv, dk, static_cast<const __nv_bfloat16 *>(wk), wk_stride, kt};
+    const dim3 pg((nb + kProjRows - 1) / kProjRows, B * (Hq + Hkv));
+    project_rope_kernel<<<pg, kProjThreads, psmem, stream>>>(jq, jk, B * Hq, nb, nb, dg, (double)theta, 0);
     e = cudaGetLastError();
     if (e != cudaSuccess)
         return e;
     const size_t ssmem = sizeof(float) * (size_t)(kLR + kLC) * (dg + kLPad);
-    e = cudaFuncSetAttribute(gate_softmax_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ssmem);
+    const bool pf = kLC * (dg / 4) <= kLPF * kLThreads;
+    e = cudaFuncSetAttribute(pf ? gate_softmax_kernel<true> : gate_softmax_kernel<false>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ssmem);
     if (e != cudaSuccess)
         return e;
     const dim3 sg(B * Hq, (nb + kLR - 1) / kLR);
-    gate_softmax_kernel<<<sg, kLThreads, ssmem, stream>>>(qt, kt, Hq, Hkv, nb, dg, 1.0f / sqrtf((float)dg), scores);
+    if (pf)
+        gate_softmax_kernel<true><<<sg, kLThreads, ssmem, stream>>>(qt, kt, Hq, Hkv, nb, dg, 1.0f / sqrtf((float)dg),
+                                                                   scores);
+    else
+        gate_softmax_kernel<false><<<sg, kLThreads, ssmem, stream>>>(qt, kt, Hq, Hkv, nb, dg, 1.0f / sqrtf((float)dg),
+                                                                    scores);
     return cudaGetLastError();
 }
 
@@ -531,9 +599,10 @@ cudaError_t launch_gate_keys(int B, int Hkv, int L, int d, int dg, float theta, 
     e = cudaFuncSetAttribute(project_rope_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)psmem);
     if (e != cudaSuccess)
         return e;
+    const ProjJob jk{kp + (size_t)first_block * dk, Hkv, dk, static_cast<const __nv_bfloat16 *>(wk), wk_stride,
+                     kt + (size_t)first_block * dg};
     project_rope_kernel<<<dim3((nsel + kProjRows - 1) / kProjRows, B * Hkv), kProjThreads, psmem, stream>>>(
-        kp + (size_t)first_block * dk, Hkv, nsel, nb, dk, static_cast<const __nv_bfloat16 *>(wk), wk_stride, dg,
-        (double)theta, first_block, kt + (size_t)first_block * dg);
+        jk, jk, B * Hkv, nsel, nb, dg, (double)theta, first_block);
     return cudaGetLastError();
 }
 
@@ -553,8 +622,9 @@ cudaError_t launch_decode_gate_cached(int B, int Hq, int Hkv, int L, int d, int 
     if (e != cudaSuccess)
         return e;
     // the token's q: one row per head, rotated at its block, nb - 1
-    project_rope_kernel<<<dim3(1, B * Hq), kProjThreads, psmem_q, stream>>>(
-        qp, Hq, 1, 1, d, static_cast<const __nv_bfloat16 *>(wq), wq_stride, dg, (double)theta, nb - 1, qt);
+    const ProjJob jq{qp, Hq, d, static_cast<const __nv_bfloat16 *>(wq), wq_stride, qt};
+    project_rope_kernel<<<dim3(1, B * Hq), kProjThreads, psmem_q, stream>>>(jq, jq, B * Hq, 1, 1, dg, (double)theta,
+                                                                         nb - 1);
     e = cudaGetLastError();
     if (e != cudaSuccess)
         return e;
