@@ -632,3 +632,46 @@ def test_decode_attention_brute_force(oracle, L):
     p = np.exp(s - s.max(-1, keepdims=True))
     np.testing.assert_allclose(o1[0], np.einsum("hc,hcd->hd", p, np.repeat(v[0], 2, axis=0)) / p.sum(-1, keepdims=True),
                                rtol=1e-10, atol=1e-12)
+
+
+# ------------------------------------------------- pooling: shapes and torch
+def _golden_rows(name):
+    import os
+    path = os.path.join(os.path.dirname(__file__), "golden", name)
+    rows = []
+    for line in open(path):
+        line = line.split("#", 1)[0].strip()
+        if line:
+            lhs, rhs = line.split("->")
+            rows.append((lhs.split(), tuple(int(v) for v in rhs.split())))
+    return rows
+
+
+def test_pool_shapes_golden(oracle):
+    """Worked shape example of the pooling (rebuttal, Weakness 3 and 4)."""
+    rows = _golden_rows("pooling_shapes.txt")
+    assert len(rows) >= 5
+    for (b, h, s, d, kind), want in rows:
+        bits = rand_bits((int(b), int(h), int(s), int(d)), 7)
+        out = oracle.pool_avg(bits) if kind == "avg" else oracle.pool_maxmin(bits)
+        assert out.shape == want, (b, h, s, d, kind)
+
+
+def test_pool_matches_torch_ceil_mode(oracle):
+    """Rebuttal, Weakness 4: ragged sequences pool like torch's pooling with
+    ceil_mode=True (the window past the end covers only the real tokens)."""
+    torch = pytest.importorskip("torch")
+    F = torch.nn.functional
+    for S in (BLOCK, 2 * BLOCK + 1, 3 * BLOCK + 40, 5 * BLOCK - 1):
+        bits = rand_bits((2, 3, S, 8), 200 + S)
+        x = torch.from_numpy(bits_to_f64(bits))                      # [B, H, S, d]
+        xs = x.permute(0, 1, 3, 2).reshape(-1, 1, S)                 # pool along S
+        avg = F.avg_pool1d(xs, BLOCK, BLOCK, ceil_mode=True)
+        mx = F.max_pool1d(xs, BLOCK, BLOCK, ceil_mode=True)
+        mn = -F.max_pool1d(-xs, BLOCK, BLOCK, ceil_mode=True)
+        nb = -(-S // BLOCK)
+        to4 = lambda t: t.reshape(2, 3, 8, nb).permute(0, 1, 3, 2).numpy()
+        np.testing.assert_allclose(oracle.pool_avg(bits), to4(avg), rtol=0, atol=1e-14)
+        mm = oracle.pool_maxmin(bits)
+        np.testing.assert_array_equal(mm[..., :8], to4(mx))
+        np.testing.assert_array_equal(mm[..., 8:], to4(mn))
