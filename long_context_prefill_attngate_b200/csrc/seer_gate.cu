@@ -126,9 +126,23 @@ constexpr int kPA = kProjRows / 16;         // rows per thread
 constexpr int kProjThreads = 256;      // 16 x 16: rows ty + 16a, rotation pairs tx + 16b
 constexpr int kPStride = 4;            // padding (floats) of the shared rows
 
+// d = a * b + c on a pair of floats in one packed instruction (sm_100); each
+// half is rounded exactly like fmaf.
+__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c)
+{
+    float2 d;
+    asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
+        "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rc, {%6, %7};\n\t"
+        "fma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(d.x), "=f"(d.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+    return d;
+}
+
 // out[bh, i, :] = RoPE_{pos0+i}( xp[bh, i, :] @ W[h] ) for i < nb (rows ld apart
 // between heads), kProjRows rows i of one
-// head.  Each thread owns kPA rows x 4 rotation pairs (t, t + dg/2), so both halves
+// head.  Each thread owns kPA rows x 4 rotation pairs (t, t + dg/2) — two
+// adjacent column pairs, multiplied with packed fp32 FMAs — so both halves
 // of a pair are in its registers when the rotation is applied.  Angles
 // i * theta^(-2t/dg): frequencies in double once per CTA, angle formed and
 // reduced modulo 2*pi in double, the reduced angle through fp32 sincosf.
@@ -192,33 +206,41 @@ __global__ void __launch_bounds__(kProjThreads)
     constexpr double kTwoPi = 6.283185307179586476925286766559;
     const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
     for (int t0 = 0; t0 < half; t0 += 64) {
-        float y0[kPA][4], y1[kPA][4];
+        // columns (tcol[q], tcol[q] + 1), q = 0, 1; dg and half are even, so a
+        // pair lies wholly inside [0, half) or wholly outside it
+        int tcol[2];
+        bool tok[2];
+#pragma unroll
+        for (int q = 0; q < 2; ++q) {
+            tcol[q] = t0 + 32 * q + 2 * tx;
+            tok[q] = tcol[q] < half;
+            if (!tok[q])
+                tcol[q] = 0;
+        }
+        float2 y0[kPA][2], y1[kPA][2];
 #pragma unroll
         for (int a = 0; a < kPA; ++a)
 #pragma unroll
-            for (int b = 0; b < 4; ++b)
-                y0[a][b] = y1[a][b] = 0.f;
-        int tcol[4];
-#pragma unroll
-        for (int b = 0; b < 4; ++b)
-            tcol[b] = min(t0 + tx + 16 * b, half - 1);
+            for (int q = 0; q < 2; ++q)
+                y0[a][q] = y1[a][q] = make_float2(0.f, 0.f);
 #pragma unroll 2
         for (int c = 0; c < d; ++c) {
-            float xv[kPA], w0[4], w1[4];
+            float xv[kPA];
+            float2 w0[2], w1[2];
 #pragma unroll
             for (int a = 0; a < kPA; ++a)
                 xv[a] = sx[(ty + 16 * a) * xs + c];
 #pragma unroll
-            for (int b = 0; b < 4; ++b) {
-                w0[b] = sw[c * dg + tcol[b]];
-                w1[b] = sw[c * dg + tcol[b] + half];
+            for (int q = 0; q < 2; ++q) {
+                w0[q] = *reinterpret_cast<const float2 *>(sw + c * dg + tcol[q]);
+                w1[q] = *reinterpret_cast<const float2 *>(sw + c * dg + tcol[q] + half);
             }
 #pragma unroll
             for (int a = 0; a < kPA; ++a)
 #pragma unroll
-                for (int b = 0; b < 4; ++b) {
-                    y0[a][b] = fmaf(xv[a], w0[b], y0[a][b]);
-                    y1[a][b] = fmaf(xv[a], w1[b], y1[a][b]);
+                for (int q = 0; q < 2; ++q) {
+                    y0[a][q] = fma2(make_float2(xv[a], xv[a]), w0[q], y0[a][q]);
+                    y1[a][q] = fma2(make_float2(xv[a], xv[a]), w1[q], y1[a][q]);
                 }
         }
 #pragma unroll
@@ -230,15 +252,18 @@ __global__ void __launch_bounds__(kProjThreads)
             float *o = out + ((long long)bh * ld + i) * dg;
 #pragma unroll
             for (int b = 0; b < 4; ++b) {
-                const int t = t0 + tx + 16 * b;
-                if (t >= half)
+                const int q = b >> 1;
+                if (!tok[q])
                     continue;
+                const int t = tcol[q] + (b & 1);
+                const float v0 = (b & 1) ? y0[a][q].y : y0[a][q].x;
+                const float v1 = (b & 1) ? y1[a][q].y : y1[a][q].x;
                 const double ang = (double)(pos0 + i) * sfreq[t];
                 const double red = ang - rint(ang * (1.0 / kTwoPi)) * kTwoPi;
                 float sn, cs;
                 sincosf((float)red, &sn, &cs);
-                o[t] = y0[a][b] * cs - y1[a][b] * sn;
-                o[t + half] = y1[a][b] * cs + y0[a][b] * sn;
+                o[t] = v0 * cs - v1 * sn;
+                o[t + half] = v1 * cs + v0 * sn;
             }
         }
     }
