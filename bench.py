@@ -402,7 +402,7 @@ def run_gpu(args, world, rank, local):
     # mask reads the causal scores and writes the mask.
     gate_bytes = 2 * (w.B * w.Hq * w.S * w.d + w.B * w.Hkv * w.S * w.d) + 4 * w.B * w.Hq * nb * nb
     mask_bytes = 4 * w.B * w.Hq * nb * (nb + 1) // 2 + w.B * w.Hq * nb * nb
-    launches_per_step = 5 + 1 + 1   # gate: 2 pool + 2 project/RoPE + 1 softmax; mask: 1; attention: 1
+    launches_per_step, launches_src = count_step_launches(lambda: (gate_mask(args.density), attention()))
     out = {
         "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms_step_max, 4), "higher_is_better": True,
@@ -428,10 +428,28 @@ def run_gpu(args, world, rank, local):
         "e2e": None if e2e_value is None else {"value": round(e2e_value, 2), "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 3)},
         "gpu_launches": launches_per_step * args.steps,
+        "gpu_launches_per_step": {"count": launches_per_step, "source": launches_src},
         "clocks": clocks, "cpu_baseline": cpu_baseline, "wall_s_timed_region": round(t_wall, 3),
     }
     if rank == 0:
         print(json.dumps(out), flush=True)
+
+
+def count_step_launches(step_fn):
+    """Kernels of this library that one step launches, counted from the CUDA
+    activity trace of one extra (untimed) step."""
+    import torch
+    from torch.profiler import ProfilerActivity, profile
+
+    try:
+        torch.cuda.synchronize()
+        with profile(activities=[ProfilerActivity.CUDA]) as prof:
+            step_fn()
+            torch.cuda.synchronize()
+        n = sum(ev.count for ev in prof.key_averages() if "seer::" in ev.key and ev.device_time_total > 0)
+        return n, "cuda activity trace of one step (kernels in namespace seer)"
+    except Exception as exc:   # the profiler is optional; the count is then the static one
+        return 5, f"static count (gate 3 + mask 1 + attention 1); trace unavailable: {exc!r}"[:200]
 
 
 def oracle_sample(w, x, mask_np, budget_s: float):
