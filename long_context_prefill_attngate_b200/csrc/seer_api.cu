@@ -21,6 +21,12 @@ namespace seer {
 // pointer (first error wins); seer_check_status() reads and clears it.
 __device__ int g_status_word;
 
+// Tile counters of the attention launches: a ring per device, one slot per
+// launch, zeroed on the launch stream.  256 launches can be in flight at once
+// (on any number of streams) before a slot is reused.
+constexpr int kTileCounterRing = 256;
+__device__ unsigned long long g_tile_counters[kTileCounterRing];
+
 namespace {
 
 thread_local char g_err[512] = "";
@@ -82,6 +88,37 @@ int *status_ptr()
         cache[dev] = static_cast<int *>(p);
     }
     return cache[dev];
+}
+
+// A tile counter for one attention launch: the next slot of this device's
+// ring, zeroed on `stream` before the launch.  Null on a CUDA error (in *err).
+unsigned long long *tile_counter(cudaStream_t stream, cudaError_t *err)
+{
+    static std::mutex mu;
+    static unsigned long long *cache[64] = {nullptr};
+    static unsigned next[64] = {0};
+    int dev = 0;
+    *err = cudaGetDevice(&dev);
+    if (*err != cudaSuccess)
+        return nullptr;
+    if (dev < 0 || dev >= 64) {
+        *err = cudaErrorInvalidDevice;
+        return nullptr;
+    }
+    unsigned long long *c = nullptr;
+    {
+        std::lock_guard<std::mutex> lk(mu);
+        if (cache[dev] == nullptr) {
+            void *ptr = nullptr;
+            *err = cudaGetSymbolAddress(&ptr, g_tile_counters);
+            if (*err != cudaSuccess)
+                return nullptr;
+            cache[dev] = static_cast<unsigned long long *>(ptr);
+        }
+        c = cache[dev] + (next[dev]++ % kTileCounterRing);
+    }
+    *err = cudaMemsetAsync(c, 0, sizeof(unsigned long long), stream);
+    return *err == cudaSuccess ? c : nullptr;
 }
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
@@ -331,7 +368,11 @@ seer_status seer_block_sparse_prefill(const seer_shape *shape, const void *q, co
     a.map_mode = false;
     a.timeout_ns = g_timeout_ns;
     a.status = status;
-    const cudaError_t e = launch_attention(a, static_cast<cudaStream_t>(stream));
+    cudaError_t e = cudaSuccess;
+    a.tile_ctr = tile_counter(static_cast<cudaStream_t>(stream), &e);
+    if (a.tile_ctr == nullptr)
+        return cuda_fail(e, "seer_block_sparse_prefill tile counter");
+    e = launch_attention(a, static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess)
         return cuda_fail(e, "seer_block_sparse_prefill launch");
     return ok();
@@ -378,6 +419,9 @@ seer_status seer_attn_pooled_map(const seer_shape *shape, const void *q, const v
     a.map_mode = true;
     a.timeout_ns = g_timeout_ns;
     a.status = status;
+    a.tile_ctr = tile_counter(s, &e);
+    if (a.tile_ctr == nullptr)
+        return cuda_fail(e, "seer_attn_pooled_map tile counter");
     e = launch_attention(a, s);
     if (e != cudaSuccess)
         return cuda_fail(e, "seer_attn_pooled_map launch");

@@ -31,6 +31,7 @@ struct AttnLaunch {
     bool map_mode;
     uint64_t timeout_ns;
     int *status;                  // device status word
+    unsigned long long *tile_ctr; // tile counter of this launch, zeroed on the launch stream
 };
 
 // Attention kernels (seer_attn.cu).  Returns a cudaError_t.
