@@ -212,6 +212,40 @@ def test_prefill_repeatable():
     assert torch.equal(o1, o2)
 
 
+def test_prefill_concurrent_streams_and_counter_ring():
+    """Launches on different streams take tiles from different counters: two
+    concurrent calls give exactly their one-at-a-time results, and more calls
+    than the counter ring holds (256) in a row stay exact."""
+    w1 = syn.custom("cs1", 1, 8, 2, 4096, 128, number=41)
+    w2 = syn.custom("cs2", 2, 4, 1, 2048, 64, number=42)
+    x1, x2 = syn.make_inputs(w1), syn.make_inputs(w2)
+    m1 = dev(syn.random_mask(1, 8, 64, 0.3, seed=43))
+    m2 = dev(syn.random_mask(2, 4, 32, 0.5, seed=44))
+    a = [dev(x1[n]) for n in ("q", "k", "v")]
+    b = [dev(x2[n]) for n in ("q", "k", "v")]
+    ref1 = seer.seer_block_sparse_prefill(*a, m1)
+    ref2 = seer.seer_block_sparse_prefill(*b, m2)
+    torch.cuda.synchronize()
+    s1, s2 = torch.cuda.Stream(), torch.cuda.Stream()
+    o1, o2 = torch.empty_like(ref1), torch.empty_like(ref2)
+    for _ in range(5):
+        o1.zero_()
+        o2.zero_()
+        torch.cuda.synchronize()
+        with torch.cuda.stream(s1):
+            seer.seer_block_sparse_prefill(*a, m1, o=o1, stream=s1)
+        with torch.cuda.stream(s2):
+            seer.seer_block_sparse_prefill(*b, m2, o=o2, stream=s2)
+        torch.cuda.synchronize()
+        assert torch.equal(o1, ref1) and torch.equal(o2, ref2)
+    o = torch.empty_like(ref2)
+    for _ in range(300):
+        seer.seer_block_sparse_prefill(*b, m2, o=o)
+    torch.cuda.synchronize()
+    seer.seer_check_status()
+    assert torch.equal(o, ref2)
+
+
 def test_prefill_max_sequence(oracle):
     """S = 2^20 (the largest nb the library accepts): first + diagonal blocks only."""
     B, Hq, Hkv, S, d = 1, 2, 1, 1 << 20, 64
