@@ -170,6 +170,12 @@ SEER_API seer_status seer_compact_mask(const seer_shape *shape, const uint8_t *m
  * softmax_scale <= 0 selects 1/sqrt(d).  q, k, v, o must be 16-B aligned.
  * Workspace: seer_workspace_bytes(SEER_CALL_BLOCK_SPARSE_PREFILL) (may be 0;
  * workspace may then be NULL).
+ * Scheduling: the persistent grid's tile slots take tiles from a counter
+ * that the call zeroes on `stream` (an 8-byte memset before the launch);
+ * counters come from a per-device ring of 256, so up to 256 prefill / pooled-
+ * map launches may be in flight at once on any streams.  A CUDA graph that
+ * captured the call reuses its counter on every replay, so one graph must
+ * not be replayed on two streams at once.
  */
 SEER_API seer_status seer_block_sparse_prefill(const seer_shape *shape, const void *q, const void *k,
                                       const void *v, const uint8_t *mask, float softmax_scale,
@@ -185,7 +191,8 @@ SEER_API seer_status seer_block_sparse_prefill(const seer_shape *shape, const vo
  * with P the causal softmax of scale * q.k.  A is not row-normalised.
  * q/k/v/o as above; A: fp32 [B,Hq,nb,nb] (fully written).  Workspace:
  * seer_workspace_bytes(SEER_CALL_ATTN_POOLED_MAP, shape) bytes (holds the
- * per-row block maxima of the queries in flight).
+ * per-row block maxima of the queries in flight).  Tiles are scheduled as in
+ * seer_block_sparse_prefill (same counter ring and limits).
  */
 SEER_API seer_status seer_attn_pooled_map(const seer_shape *shape, const void *q, const void *k,
                                  const void *v, float softmax_scale, void *o, float *A,
