@@ -31,7 +31,8 @@
  *    seer_check_status().
  *  - seer_last_error() returns a thread-local text for the last failure.
  *  - Supported: any S >= 1 with nb = ceil(S/64) <= 16384, d in {64, 128},
- *    Hq % Hkv == 0.  Other shapes return SEER_ERR_UNSUPPORTED.
+ *    Hq % Hkv == 0, B * Hq <= 65535.  Other shapes return
+ *    SEER_ERR_UNSUPPORTED.
  *  - S not a multiple of 64 ("Learning Intrinsic Sparse Attention",
  *    rebuttal Weakness 4: padding, ceil-mode pooling): the last block holds
  *    the S - 64 (nb - 1) remaining tokens; it pools only those tokens, and no

@@ -65,8 +65,10 @@ seer_status check_shape(const seer_shape *sh)
         return fail(SEER_ERR_UNSUPPORTED, "head dim %d not supported (64 or 128)", sh->d);
     if (num_blocks(sh->S) > kMaxNb)
         return fail(SEER_ERR_UNSUPPORTED, "ceil(S/64) = %d exceeds %d", num_blocks(sh->S), kMaxNb);
-    if ((long long)sh->B * sh->Hq > (1LL << 30) / kMaxNb)
-        return fail(SEER_ERR_UNSUPPORTED, "B*Hq too large");
+    // B*Hq and B*Hkv index a grid dimension of at most 65535 in the decode and
+    // gate kernels (and B*Hq*nb stays below 2^30).
+    if ((long long)sh->B * sh->Hq > 65535)
+        return fail(SEER_ERR_UNSUPPORTED, "B*Hq = %lld exceeds 65535", (long long)sh->B * sh->Hq);
     return SEER_OK;
 }
 

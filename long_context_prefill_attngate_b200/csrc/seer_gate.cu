@@ -154,14 +154,15 @@ struct ProjJob {
     float *out;                      // [B*H, ld, dg]
 };
 
-// Two projections in one launch: grid rows blockIdx.y < ny0 run job j0, the
-// rest job j1 (the Q and K sides of the gate, which would otherwise leave
-// most of the GPU idle in the smaller launch).
+// Two projections in one launch (the Q and K sides of the gate: the K grid
+// alone would leave most of the GPU idle): blockIdx.x < ny0 is head row
+// blockIdx.x of job j0, the rest are job j1's; blockIdx.y is the chunk of
+// kProjRows blocks.
 __global__ void __launch_bounds__(kProjThreads)
     project_rope_kernel(ProjJob j0, ProjJob j1, int ny0, int nb, int ld, int dg, double theta, int pos0)
 {
     extern __shared__ float4 psm4[];
-    const bool second = (int)blockIdx.y >= ny0;
+    const bool second = (int)blockIdx.x >= ny0;
     const ProjJob &job = second ? j1 : j0;
     const float *__restrict__ xp = job.xp;
     const int H = job.H, d = job.d;
@@ -172,9 +173,9 @@ __global__ void __launch_bounds__(kProjThreads)
     float *sx = reinterpret_cast<float *>(psm4);           // kProjRows x xs
     float *sw = sx + kProjRows * xs;                       // d x dg (fp32)
     double *sfreq = reinterpret_cast<double *>(sw + d * dg);
-    const int bh = (int)blockIdx.y - (second ? ny0 : 0);
+    const int bh = (int)blockIdx.x - (second ? ny0 : 0);
     const int h = bh % H;
-    const int i0 = blockIdx.x * kProjRows;
+    const int i0 = blockIdx.y * kProjRows;
     const int rows = min(kProjRows, nb - i0);
     const int half = dg / 2;
     const __nv_bfloat16 *wh = w + (long long)h * w_stride;
@@ -563,7 +564,7 @@ cudaError_t launch_gate(int B, int Hq, int Hkv, int S, int d, int dg, float thet
         return e;
     const ProjJob jq{qp, Hq, d, static_cast<const __nv_bfloat16 *>(wq), wq_stride, qt};
     const ProjJob jk{kp, Hkv, dk, static_cast<const __nv_bfloat16 *>(wk), wk_stride, kt};
-    const dim3 pg((nb + kProjRows - 1) / kProjRows, B * (Hq + Hkv));
+    const dim3 pg(B * (Hq + Hkv), (nb + kProjRows - 1) / kProjRows);
     project_rope_kernel<<<pg, kProjThreads, psmem, stream>>>(jq, jk, B * Hq, nb, nb, dg, (double)theta, 0);
     e = cudaGetLastError();
     if (e != cudaSuccess)
@@ -626,7 +627,7 @@ cudaError_t launch_gate_keys(int B, int Hkv, int L, int d, int dg, float theta, 
         return e;
     const ProjJob jk{kp + (size_t)first_block * dk, Hkv, dk, static_cast<const __nv_bfloat16 *>(wk), wk_stride,
                      kt + (size_t)first_block * dg};
-    project_rope_kernel<<<dim3((nsel + kProjRows - 1) / kProjRows, B * Hkv), kProjThreads, psmem, stream>>>(
+    project_rope_kernel<<<dim3(B * Hkv, (nsel + kProjRows - 1) / kProjRows), kProjThreads, psmem, stream>>>(
         jk, jk, B * Hkv, nsel, nb, dg, (double)theta, first_block);
     return cudaGetLastError();
 }
@@ -648,7 +649,7 @@ cudaError_t launch_decode_gate_cached(int B, int Hq, int Hkv, int L, int d, int 
         return e;
     // the token's q: one row per head, rotated at its block, nb - 1
     const ProjJob jq{qp, Hq, d, static_cast<const __nv_bfloat16 *>(wq), wq_stride, qt};
-    project_rope_kernel<<<dim3(1, B * Hq), kProjThreads, psmem_q, stream>>>(jq, jq, B * Hq, 1, 1, dg, (double)theta,
+    project_rope_kernel<<<dim3(B * Hq, 1), kProjThreads, psmem_q, stream>>>(jq, jq, B * Hq, 1, 1, dg, (double)theta,
                                                                          nb - 1);
     e = cudaGetLastError();
     if (e != cudaSuccess)

@@ -56,6 +56,7 @@ def test_workspace_sizes(L):
     ((1, 30, 8, 4096, 128), seer.SEER_ERR_INVALID_ARG, "multiple of Hkv"),
     ((0, 32, 8, 4096, 128), seer.SEER_ERR_INVALID_ARG, "positive"),
     ((1, 2, 2, 64 * 20000, 64), seer.SEER_ERR_UNSUPPORTED, "exceeds"),
+    ((2048, 32, 8, 64, 64), seer.SEER_ERR_UNSUPPORTED, "exceeds 65535"),
 ])
 def test_shape_rejections(L, shape, status, msg):
     sh = seer.seer_shape(*shape)
