@@ -518,9 +518,14 @@ def oracle_sample(w, x, mask_np, budget_s: float):
             break
     cores = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
     n = sum(len(u) for u in units)
+    # the oracle's gate (a1-a3) in full on the same layer, timed on its own
+    t = time.time()
+    oracle.gate_scores(qb, kb, syn.bf16_bits(x["wq"]), syn.bf16_bits(x["wk"]), theta=w.rope_theta)
+    gate_s = time.time() - t
     return {"value": flops / spent / 1e12, "unit": UNIT, "cores": cores, "kind": "oracle",
             "sample": f"{n} random (head, query block) units of {w.name} at the benchmark mask "
-                      f"(fp64 masked attention, {spent:.1f} s; gate/mask not included)"}
+                      f"(fp64 masked attention, {spent:.1f} s; gate/mask not included)",
+            "gate_full_layer_s": round(gate_s, 3)}
 
 
 # --------------------------------------------------------------------------- reference arm
