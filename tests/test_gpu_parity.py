@@ -530,3 +530,50 @@ def test_host_prefill_matches_whole_layer_calls(oracle, B, Hq, Hkv, S, d):
     torch.cuda.synchronize()
     assert torch.equal(hp.mask.cpu(), m.cpu())
     assert torch.equal(ho, o.cpu())
+
+
+# ------------------------------------------------------------------ every output element written
+def test_outputs_fully_written_over_poison():
+    """Outputs pre-filled with NaN (0xFF for the mask) come back finite and equal
+    to the results of calls on zero-filled outputs: no tile, row or tail block of
+    any output is left unwritten (ragged S, GQA, decode included)."""
+    B, Hq, Hkv, S, d = 1, 4, 2, 7 * BLOCK + 29, 128
+    nb = -(-S // BLOCK)
+    w = syn.custom("poison", B, Hq, Hkv, S, d, number=431)
+    x = syn.make_inputs(w)
+    q, k, v, wq, wk = (dev(x[n]) for n in ("q", "k", "v", "wq", "wk"))
+    nan = float("nan")
+
+    s_p = torch.full((B, Hq, nb, nb), nan, dtype=torch.float32, device="cuda")
+    seer.seer_gate_scores(q, k, wq, wk, rope_theta=w.rope_theta, scores=s_p)
+    s_z = seer.seer_gate_scores(q, k, wq, wk, rope_theta=w.rope_theta)
+    m_p = torch.full((B, Hq, nb, nb), 255, dtype=torch.uint8, device="cuda")
+    seer.seer_block_mask(s_z, "topk", density=0.3, mask=m_p, Hkv=Hkv, d=d)
+    m_z = seer.seer_block_mask(s_z, "topk", density=0.3, Hkv=Hkv, d=d)
+    o_p = torch.full_like(q, nan)
+    lse_p = torch.full((B, Hq, S), nan, dtype=torch.float32, device="cuda")
+    seer.seer_block_sparse_prefill(q, k, v, m_z, o=o_p, lse=lse_p)
+    o_z, lse_z = seer.seer_block_sparse_prefill(q, k, v, m_z, return_lse=True)
+    om_p = torch.full_like(q, nan)
+    A_p = torch.full((B, Hq, nb, nb), nan, dtype=torch.float32, device="cuda")
+    seer.seer_attn_pooled_map(q, k, v, o=om_p, A=A_p)
+    om_z, A_z = seer.seer_attn_pooled_map(q, k, v)
+    q_tok = q[:, :, -1].contiguous()
+    ds = seer.seer_decode_gate_scores(q_tok, k, wq, wk, rope_theta=w.rope_theta)
+    dm = seer.seer_decode_block_mask(ds, "topk", density=0.3)
+    do_p = torch.full_like(q_tok, nan)
+    dl_p = torch.full((B, Hq), nan, dtype=torch.float32, device="cuda")
+    seer.seer_block_sparse_decode(q_tok, k, v, dm, o=do_p, lse=dl_p)
+    do_z, dl_z = seer.seer_block_sparse_decode(q_tok, k, v, dm, return_lse=True)
+    torch.cuda.synchronize()
+    seer.seer_check_status()
+
+    assert torch.isfinite(s_p).all() and torch.equal(s_p, s_z)
+    assert int(m_p.max()) <= 1 and torch.equal(m_p, m_z)
+    assert not torch.triu(m_p.view(-1, nb, nb).to(torch.int32), diagonal=1).any()
+    assert torch.isfinite(o_p.float()).all() and torch.equal(o_p, o_z)
+    assert torch.isfinite(lse_p).all() and torch.equal(lse_p, lse_z)
+    assert torch.isfinite(om_p.float()).all() and torch.equal(om_p, om_z)
+    assert torch.isfinite(A_p).all() and torch.equal(A_p, A_z)
+    assert torch.isfinite(do_p.float()).all() and torch.equal(do_p, do_z)
+    assert torch.isfinite(dl_p).all() and torch.equal(dl_p, dl_z)
