@@ -6,15 +6,18 @@ attention (GQA).  Default workload: Llama-3.1-8B-shaped layer (32 q-heads,
 8 kv-heads, head dim 128) at 32k tokens, TopK density 0.1 (first and diagonal
 blocks kept).  Reported value: active-block TFLOP/s of the whole step
 (4*64*64*d flops per active (head, query block, key block)), summed over ranks
-(weak scaling: every rank runs its own layer) over the max time across ranks.
+over the max time across ranks.  With N ranks, either every rank runs its own
+layer (--split replicas, weak scaling) or the ranks split one layer by KV-head
+group (--split heads, strong scaling; no collective on the data path).
 
-  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference] [--split heads]
 
 Prints ONE JSON line on rank 0.
 """
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import hashlib
 import json
 import math
@@ -147,6 +150,17 @@ def max_over_ranks(x: float, world: int) -> float:
     return float(t.item())
 
 
+def sum_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
 def barrier(world: int):
     if world > 1:
         import torch.distributed as dist
@@ -162,11 +176,20 @@ def run_gpu(args, world, rank, local):
     from long_context_prefill_attngate_b200 import build as seer_build
     from long_context_prefill_attngate_b200 import synthetic as syn
 
+    from long_context_prefill_attngate_b200 import partition
+
     seer_build.build()
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
-    w = syn.WORKLOADS[args.workload]
-    x = syn.make_inputs(w, seed=w.seed + 1000 * rank)
+    w_full = syn.WORKLOADS[args.workload]
+    if args.split == "heads" and world > 1:
+        # One layer split by KV-head group: every rank draws the same layer and keeps its heads.
+        x = partition.slice_layer(syn.make_inputs(w_full), w_full.Hq, w_full.Hkv, world, rank)
+        q0, q1, k0, k1 = partition.head_range(w_full.Hq, w_full.Hkv, world, rank)
+        w = dataclasses.replace(w_full, Hq=q1 - q0, Hkv=k1 - k0)
+    else:
+        x = syn.make_inputs(w_full, seed=w_full.seed + 1000 * rank)
+        w = w_full
     pk, pk_kind = peaks()
     stream = torch.cuda.current_stream()
 
@@ -227,14 +250,32 @@ def run_gpu(args, world, rank, local):
     clocks = clk.summary()
     mask_sum = int(mask.sum(dtype=torch.int64).item())
     flops = attn_flops(mask_sum, w.d)
+    flops_all = sum_over_ranks(flops, world)          # work of all ranks (replicas or head slices)
     density_meas = mask_sum / (w.B * w.Hq * nb * (nb + 1) / 2)
     ms_step = statistics.mean(res["step"])
     ms_attn = statistics.mean(res["attn"])
     ms_gate = statistics.mean(res["gate"])
     ms_mask = statistics.mean(res["mask"])
     ms_step_max = max_over_ranks(ms_step, world)
-    value = world * flops / (ms_step_max * 1e-3) / 1e12
+    value = flops_all / (ms_step_max * 1e-3) / 1e12
     attn_tflops = flops / (ms_attn * 1e-3) / 1e12
+
+    # ---------------- steady state: the same step back to back for about a second
+    # (L2 flushed before every step, outside its events), with its own clock record,
+    # so the headline can be read against a power-capped steady state.
+    steady = None
+    if args.steady_steps > 0:
+        with ClockSampler(local) as clk2:
+            t0 = time.time()
+            r2 = timed_steps(args.density, args.steady_steps, 0)
+            wall2 = time.time() - t0
+        a2 = statistics.mean(r2["attn"])
+        st2 = max_over_ranks(statistics.mean(r2["step"]), world)
+        steady = {"steps": args.steady_steps, "wall_s": round(wall2, 3), "ms_per_step": round(st2, 4),
+                  "value": round(flops_all / (st2 * 1e-3) / 1e12, 2), "ms_layer_attention": round(a2, 4),
+                  "attention_active_tflops": round(flops / (a2 * 1e-3) / 1e12, 1),
+                  "frac_of_bf16_peak": round(flops / (a2 * 1e-3) / 1e12 / pk["bf16_tflops"], 4),
+                  "clocks": clk2.summary()}
 
     # ---------------- density sweep (attention only; 1.0 is the dense causal point)
     sweep = []
@@ -429,29 +470,47 @@ def run_gpu(args, world, rank, local):
         barrier(world)
         seer.seer_check_status()
         e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps, world)
-        e2e_value = world * flops / (e2e_ms * 1e-3) / 1e12
+        e2e_value = flops_all / (e2e_ms * 1e-3) / 1e12
 
-    # ---------------- CPU baseline: the oracle on a bounded sample (rank 0, N=1)
+    # ---------------- host link: pinned 256 MiB copies each way (what bounds the e2e leg)
+    host_link = None
+    if not args.no_e2e:
+        host_link = measure_host_link(dev, stream)
+
+    # ---------------- CPU baseline: the oracle on a bounded sample (rank 0, N=1).  It runs in
+    # a child process that regenerates the same inputs, so this GPU process never loads the oracle.
     cpu_baseline = None
-    if rank == 0 and world == 1 and not args.no_cpu:
-        cpu_baseline = oracle_sample(w, x, mask.cpu().numpy(), budget_s=args.cpu_budget)
+    mask_np = mask.cpu().numpy() if (rank == 0 and world == 1 and not args.no_cpu) else None
 
-    traffic = profile_traffic("long_context_prefill_attngate_b200/csrc/seer_attn.cu",
+    launches_per_step, launches_src = count_step_launches(lambda: (gate_mask(args.density), attention()))
+
+    # ---------------- the other workloads of the benchmark spec, timed in the same run (N=1 only)
+    configs = None
+    if world == 1 and not args.no_configs:
+        del q, k, v, wq, wk, scores, mask, o, gws, x
+        torch.cuda.empty_cache()
+        configs = run_configs(args, dev, stream, flush, pk)
+
+    if mask_np is not None:
+        cpu_baseline = oracle_sample_subprocess(args, mask_np)
+
+    traffic = profile_traffic("long_context_prefill_attngate_b200/csrc/seer_sparse.cu",
                               "attn_sparse_llama8b_32k_d0.1.md")
     # Algorithmic bytes: gate reads Q and K once and writes the scores; the
     # mask reads the causal scores and writes the mask.
     gate_bytes = 2 * (w.B * w.Hq * w.S * w.d + w.B * w.Hkv * w.S * w.d) + 4 * w.B * w.Hq * nb * nb
     mask_bytes = 4 * w.B * w.Hq * nb * (nb + 1) // 2 + w.B * w.Hq * nb * nb
-    launches_per_step, launches_src = count_step_launches(lambda: (gate_mask(args.density), attention()))
     out = {
         "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms_step_max, 4), "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "S": w.S, "d": w.d,
-                   "mask": "gate-topk", "density_target": args.density, "density": round(density_meas, 4),
-                   "d_gate": w.d_gate, "rope_theta": w.rope_theta,
+        "scaling": "strong" if (args.split == "heads" and world > 1) else "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": w_full.name, "B": w_full.B, "Hq": w_full.Hq, "Hkv": w_full.Hkv, "S": w_full.S,
+                   "d": w_full.d, "mask": "gate-topk", "density_target": args.density,
+                   "density": round(density_meas, 4), "d_gate": w_full.d_gate, "rope_theta": w_full.rope_theta,
                    "l2": "flushed between timed steps (256 MiB write, outside the step events)",
-                   "parallelism": "replicas" if world > 1 else "single"},
+                   "parallelism": ("single" if world == 1 else
+                                   f"kv-head split x{world}" if args.split == "heads" else f"replicas x{world}")},
         "ms_layer_attention": round(ms_attn, 4), "ms_gate": round(ms_gate, 4), "ms_mask": round(ms_mask, 4),
         "gate_hbm": {"algorithmic_bytes": gate_bytes, "gbs": round(gate_bytes / (ms_gate * 1e-3) / 1e9, 1),
                      "frac_of_hbm_peak": round(gate_bytes / (ms_gate * 1e-3) / 1e9 / pk["hbm_gbs"], 4)},
@@ -462,17 +521,147 @@ def run_gpu(args, world, rank, local):
                      "unit": "TFLOP/s", "frac": round(attn_tflops / pk["bf16_tflops"], 4), "traffic": traffic,
                      "peak_kind": f"{pk_kind} bf16 burst (cuBLAS)",
                      "frac_of_sustained": round(attn_tflops / pk["bf16_tflops_sustained"], 4),
-                     "kernel": "attn_kernel<128,false> (seer_block_sparse_prefill)",
+                     "kernel": f"sparse_attn_kernel<{w.d}> (seer_block_sparse_prefill)",
                      "algorithmic_flops_per_launch": flops},
-        "density_sweep": sweep, "pooled_map": pooled, "decode": decode,
+        "steady": steady, "density_sweep": sweep, "pooled_map": pooled, "decode": decode, "configs": configs,
         "e2e": None if e2e_value is None else {"value": round(e2e_value, 2), "unit": UNIT, "h2d_bytes_per_step": h2d,
-                "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 3)},
+                "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 3), "host_link": host_link},
         "gpu_launches": launches_per_step * args.steps,
         "gpu_launches_per_step": {"count": launches_per_step, "source": launches_src},
         "clocks": clocks, "cpu_baseline": cpu_baseline, "wall_s_timed_region": round(t_wall, 3),
     }
     if rank == 0:
         print(json.dumps(out), flush=True)
+
+
+def measure_host_link(dev, stream):
+    """Pinned host <-> device copy rate (256 MiB each way, best of 3), GB/s."""
+    import torch
+    n = 256 << 20
+    h = torch.empty(n, dtype=torch.uint8).pin_memory()
+    d = torch.empty(n, dtype=torch.uint8, device=dev)
+    out = {}
+    for name, (dst, src) in (("h2d_gbs", (d, h)), ("d2h_gbs", (h, d))):
+        best = None
+        for _ in range(3):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            dst.copy_(src, non_blocking=True)
+            e1.record(stream)
+            torch.cuda.synchronize()
+            ms = e0.elapsed_time(e1)
+            best = ms if best is None else min(best, ms)
+        out[name] = round(n / (best * 1e-3) / 1e9, 1)
+    del h, d
+    return out
+
+
+def run_configs(args, dev, stream, flush, pk):
+    """Time the other workloads of the task on this GPU: the 8k threshold layer,
+    the 128k threshold layer (threshold at the 0.83 quantile of one head's causal
+    scores, for about 0.17 density) and the Qwen 64k Figure-8 pass."""
+    import torch
+
+    import long_context_prefill_attngate_b200 as seer
+    from long_context_prefill_attngate_b200 import synthetic as syn
+
+    def timed(fn, reps):
+        fn()
+        torch.cuda.synchronize()
+        ts = []
+        for _ in range(reps):
+            flush.zero_()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            fn()
+            e1.record(stream)
+            torch.cuda.synchronize()
+            ts.append(e0.elapsed_time(e1))
+        seer.seer_check_status()
+        return statistics.median(ts)
+
+    out = {}
+    for name in ("llama8b_8k", "llama8b_128k", "qwen14b_64k_map"):
+        w = syn.WORKLOADS[name]
+        x = syn.make_inputs(w)
+        q, k, v = (x[n].to(dev) for n in ("q", "k", "v"))
+        nb = w.nb
+        sh = seer.shape_of(q, k)
+        o = torch.empty_like(q)
+        if w.mask_source == "dense-map":
+            A = torch.empty((w.B, w.Hq, nb, nb), dtype=torch.float32, device=dev)
+            ws = torch.empty(seer.seer_workspace_bytes(seer.SEER_CALL_ATTN_POOLED_MAP, sh), dtype=torch.uint8,
+                             device=dev)
+            ms = timed(lambda: seer.seer_attn_pooled_map(q, k, v, o=o, A=A, workspace=ws), 3)
+            fl = attn_flops(w.B * w.Hq * nb * (nb + 1) // 2, w.d)
+            out[name] = {"pass": "Figure-8 (O and A)", "ms": round(ms, 3), "density": 1.0,
+                         "active_tflops": round(fl / (ms * 1e-3) / 1e12, 1),
+                         "frac_of_bf16_peak": round(fl / (ms * 1e-3) / 1e12 / pk["bf16_tflops"], 4),
+                         "A_bytes": A.numel() * 4}
+            del A, ws
+        else:
+            wq, wk = x["wq"].to(dev), x["wk"].to(dev)
+            gws = torch.empty(seer.seer_workspace_bytes(seer.SEER_CALL_GATE_SCORES, sh), dtype=torch.uint8,
+                              device=dev)
+            scores = torch.empty((w.B, w.Hq, nb, nb), dtype=torch.float32, device=dev)
+            mask = torch.empty((w.B, w.Hq, nb, nb), dtype=torch.uint8, device=dev)
+            ms_gate = timed(lambda: seer.seer_gate_scores(q, k, wq, wk, rope_theta=w.rope_theta, scores=scores,
+                                                           workspace=gws), 3)
+            if w.threshold is not None:
+                thr, how = w.threshold, "fixed"
+            else:
+                # the 0.83 quantile of head 0's causal scores, from an evenly strided sample
+                tri = torch.tril(torch.ones(nb, nb, dtype=torch.bool, device=dev))
+                vals = scores[0, 0][tri]
+                vals = vals[:: max(1, vals.numel() >> 20)].float()
+                thr, how = float(torch.quantile(vals, 1.0 - w.target_density)), "quantile of head 0"
+            ms_mask = timed(lambda: seer.seer_block_mask(scores, "threshold", threshold=thr, mask=mask, Hkv=w.Hkv,
+                                                         d=w.d), 3)
+            msum = int(mask.sum(dtype=torch.int64).item())
+            ms_att = timed(lambda: seer.seer_block_sparse_prefill(q, k, v, mask, o=o), 5)
+            fl = attn_flops(msum, w.d)
+            out[name] = {"mask": f"gate-threshold {thr:.4g} ({how})", "density_target": w.target_density,
+                         "density": round(msum / (w.B * w.Hq * nb * (nb + 1) / 2), 4),
+                         "ms_gate": round(ms_gate, 4), "ms_mask": round(ms_mask, 4), "ms_attention": round(ms_att, 4),
+                         "ms_layer": round(ms_gate + ms_mask + ms_att, 4),
+                         "active_tflops": round(fl / (ms_att * 1e-3) / 1e12, 1),
+                         "frac_of_bf16_peak": round(fl / (ms_att * 1e-3) / 1e12 / pk["bf16_tflops"], 4)}
+            del wq, wk, gws, scores, mask
+        del q, k, v, o, x
+        torch.cuda.empty_cache()
+    return out
+
+
+def oracle_sample_subprocess(args, mask_np):
+    """Run the CPU-baseline leg in a child process (it regenerates the same
+    inputs from the workload's seed and reads the benchmark's mask from a file)."""
+    import tempfile
+
+    import numpy as np
+    with tempfile.NamedTemporaryFile(suffix=".npy", delete=False) as f:
+        path = f.name
+    try:
+        np.save(path, mask_np)
+        cmd = [sys.executable, os.path.abspath(__file__), "--cpu-baseline-worker", path, "--workload",
+               args.workload, "--cpu-budget", str(args.cpu_budget)]
+        r = subprocess.run(cmd, capture_output=True, text=True, timeout=600)
+        lines = [ln for ln in r.stdout.splitlines() if ln.startswith("{")]
+        if r.returncode != 0 or not lines:
+            return {"unavailable": f"cpu baseline child exited {r.returncode}: {r.stderr.strip()[-200:]}"}
+        return json.loads(lines[-1])
+    finally:
+        os.unlink(path)
+
+
+def cpu_baseline_worker(args):
+    import numpy as np
+    import torch  # noqa: F401  (synthetic inputs are drawn with torch on the CPU)
+
+    from long_context_prefill_attngate_b200 import synthetic as syn
+    w = syn.WORKLOADS[args.workload]
+    x = syn.make_inputs(w)
+    mask_np = np.load(args.cpu_baseline_worker)
+    print(json.dumps(oracle_sample(w, x, mask_np, budget_s=args.cpu_budget)), flush=True)
 
 
 def count_step_launches(step_fn):
@@ -572,7 +761,11 @@ def run_reference(args, world, rank):
            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
            "data": "synthetic",
            "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "S": w.S, "d": w.d,
-                      "mask": "gate-topk", "density_target": args.density},
+                      "mask": "gate-topk", "density_target": args.density,
+                      "density": round(float(mask.sum()) / (w.B * w.Hq * w.nb * (w.nb + 1) / 2), 4),
+                      "d_gate": w.d_gate, "rope_theta": w.rope_theta,
+                      "l2": "host oracle: no GPU cache to flush",
+                      "parallelism": "single"},
            "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample},
            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(out), flush=True)
@@ -593,7 +786,15 @@ def main():
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--ref-units", type=int, default=16)
+    ap.add_argument("--split", choices=["replicas", "heads"], default="replicas",
+                    help="N>1: every rank its own layer (replicas) or one layer split by KV-head group (heads)")
+    ap.add_argument("--steady-steps", type=int, default=500, help="back-to-back steps of the steady-state block")
+    ap.add_argument("--no-configs", action="store_true", help="skip the 8k / 128k / Qwen-64k workloads")
+    ap.add_argument("--cpu-baseline-worker", default=None, help=argparse.SUPPRESS)
     args = ap.parse_args()
+    if args.cpu_baseline_worker:
+        cpu_baseline_worker(args)
+        return
     if args.warmup < 3 and args.impl == "native":
         args.warmup = 3
     world, rank, local = dist_setup(args.gpus)

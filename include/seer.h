@@ -101,6 +101,7 @@ typedef struct seer_mask_params {
                                 /*       k_per_row nor k_fixed is given             */
     int k_fixed;                /* TOPK: if > 0, k_i = k_fixed                      */
     const int32_t *k_per_row;   /* TOPK: DEVICE int32 [nb] or NULL; overrides both  */
+                                /*       (seer_topk_from_density fills a host copy) */
     int force_first;            /* keep block 0 in every row (counts toward k_i)    */
     int force_diag;             /* keep block i in row i (counts toward k_i)        */
 } seer_mask_params;
@@ -146,6 +147,22 @@ SEER_API seer_status seer_gate_scores(const seer_shape *shape, const void *q, co
  */
 SEER_API seer_status seer_block_mask(const seer_shape *shape, const float *scores,
                             const seer_mask_params *mp, uint8_t *mask, void *stream);
+
+/*
+ * seer_topk_from_density — per-row TopK counts for a target density
+ * ("Learning Intrinsic Sparse Attention", rebuttal Weakness 2: TopK is taken
+ * per query-block row).  Host function, no device work:
+ *   k_out[i] = clamp(ceil(density * (i + 1)), n_forced(i), i + 1),  0 <= i < nb,
+ * with ceil taken in double precision — the rule seer_block_mask applies on
+ * the device when it is given `density` — and n_forced(i) the blocks the flags
+ * force in row i (block 0 and the diagonal, one block in row 0).
+ * k_out: caller-owned HOST int32 [nb].  density: finite, >= 0 (values above 1
+ * give k_i = i + 1).  nb in [1, 16384].  Invalid arguments return
+ * SEER_ERR_INVALID_ARG and leave k_out untouched.  A caller that wants these
+ * counts on the device copies k_out there and passes it as k_per_row.
+ */
+SEER_API seer_status seer_topk_from_density(double density, int nb, int force_first, int force_diag,
+                                            int32_t *k_out);
 
 /*
  * seer_compact_mask — per (b, h, i) ascending list of active key blocks

@@ -17,7 +17,7 @@ from ._binding import (  # noqa: F401
     seer_decode_block_mask, seer_decode_gate_scores, seer_decode_gate_scores_cached, seer_distill_loss,
     seer_gate_key_cache, seer_gate_params, seer_gate_scores,
     seer_gate_scores_noalloc, seer_last_error, seer_mask_params, seer_set_wait_timeout_ns, seer_shape,
-    seer_version, seer_workspace_bytes, shape_of, topk_counts,
+    seer_topk_from_density, seer_version, seer_workspace_bytes, shape_of,
 )
 
 from .pipeline import HostPrefill  # noqa: F401,E402

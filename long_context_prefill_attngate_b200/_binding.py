@@ -9,7 +9,6 @@ the C entry point and raise ``SeerError`` on a non-zero status.
 from __future__ import annotations
 
 import ctypes
-import math
 import os
 import threading
 
@@ -43,7 +42,7 @@ EXPORTS = (
     "seer_attn_pooled_map", "seer_workspace_bytes", "seer_check_status", "seer_set_wait_timeout_ns",
     "seer_last_error", "seer_version", "seer_gate_scores_noalloc", "seer_distill_loss",
     "seer_decode_gate_scores", "seer_decode_block_mask", "seer_block_sparse_decode",
-    "seer_gate_key_cache", "seer_decode_gate_scores_cached",
+    "seer_gate_key_cache", "seer_decode_gate_scores_cached", "seer_topk_from_density",
 )
 
 
@@ -101,10 +100,12 @@ def lib() -> ctypes.CDLL:
             L.seer_block_sparse_decode.argtypes = [SP, P, P, P, P, F, P, P, P, Z, P]
             L.seer_gate_key_cache.argtypes = [SP, P, P, ctypes.POINTER(seer_gate_params), I, P, P, Z, P]
             L.seer_decode_gate_scores_cached.argtypes = [SP, P, P, P, ctypes.POINTER(seer_gate_params), P, P, Z, P]
+            L.seer_topk_from_density.argtypes = [ctypes.c_double, I, I, I, ctypes.POINTER(ctypes.c_int32)]
             for fn in ("seer_gate_scores", "seer_gate_scores_noalloc", "seer_block_mask", "seer_compact_mask",
                        "seer_block_sparse_prefill", "seer_attn_pooled_map", "seer_check_status",
                        "seer_distill_loss", "seer_decode_gate_scores", "seer_decode_block_mask",
-                       "seer_block_sparse_decode", "seer_gate_key_cache", "seer_decode_gate_scores_cached"):
+                       "seer_block_sparse_decode", "seer_gate_key_cache", "seer_decode_gate_scores_cached",
+                       "seer_topk_from_density"):
                 getattr(L, fn).restype = I
             L.seer_workspace_bytes.argtypes = [I, SP]
             L.seer_workspace_bytes.restype = Z
@@ -427,11 +428,9 @@ def seer_block_sparse_decode(q_tok, k, v, mask, softmax_scale: float = 0.0, o=No
     return (o, lse) if (return_lse or lse is not None) else o
 
 
-def topk_counts(density: float, nb: int, force_first: bool = True, force_diag: bool = True) -> list[int]:
-    """k_i = ceil(density*(i+1)) clamped to [forced, i+1] (host helper, same rule as the kernel)."""
-    out = []
-    for i in range(nb):
-        nf = (1 if force_first else 0) + (1 if (force_diag and not (force_first and i == 0)) else 0)
-        want = math.ceil(density * (i + 1))
-        out.append(min(max(int(min(want, i + 1)), nf), i + 1))
-    return out
+def seer_topk_from_density(density: float, nb: int, force_first: bool = True, force_diag: bool = True) -> list[int]:
+    """Per-row TopK counts k_i for a density, computed by the C library."""
+    out = (ctypes.c_int32 * nb)()
+    _check(lib().seer_topk_from_density(ctypes.c_double(float(density)), int(nb), int(bool(force_first)),
+                                        int(bool(force_diag)), out))
+    return list(out)

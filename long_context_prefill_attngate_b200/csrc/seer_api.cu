@@ -520,6 +520,29 @@ seer_status seer_decode_gate_scores_cached(const seer_shape *shape, const void *
     return ok();
 }
 
+seer_status seer_topk_from_density(double density, int nb, int force_first, int force_diag, int32_t *k_out)
+{
+    if (k_out == nullptr)
+        return fail(SEER_ERR_INVALID_ARG, "seer_topk_from_density: NULL k_out");
+    if (nb < 1 || nb > kMaxNb)
+        return fail(SEER_ERR_INVALID_ARG, "seer_topk_from_density: nb = %d outside [1, %d]", nb, kMaxNb);
+    if (!(std::isfinite(density) && density >= 0.0))
+        return fail(SEER_ERR_INVALID_ARG, "seer_topk_from_density: density must be finite and >= 0");
+    for (int i = 0; i < nb; ++i) {
+        // The rule of the TopK mask kernels: ceil(density * (i + 1)) in double,
+        // clamped to [#forced, i + 1] (block 0 and the diagonal coincide in row 0).
+        const int n_forced = (force_first ? 1 : 0) + ((force_diag && !(force_first && i == 0)) ? 1 : 0);
+        const double want = std::ceil(density * (double)(i + 1));
+        int k = want > (double)(i + 1) ? i + 1 : (int)want;
+        if (k < n_forced)
+            k = n_forced;
+        if (k > i + 1)
+            k = i + 1;
+        k_out[i] = k;
+    }
+    return ok();
+}
+
 seer_status seer_decode_block_mask(const seer_shape *shape, const float *scores, const seer_mask_params *mp,
                                    uint8_t *mask, void *stream)
 {

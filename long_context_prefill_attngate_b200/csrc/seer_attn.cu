@@ -789,6 +789,8 @@ int attn_grid_size(int B, int Hq, int Hkv, int nb)
 
 cudaError_t launch_attention(const AttnLaunch &a, cudaStream_t stream)
 {
+    if (!a.map_mode)
+        return launch_sparse_attention(a, stream);
     if (a.d == 128)
         return a.map_mode ? launch_t<128, true>(a, stream) : launch_t<128, false>(a, stream);
     if (a.d == 64)

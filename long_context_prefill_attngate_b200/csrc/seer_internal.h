@@ -36,6 +36,8 @@ struct AttnLaunch {
 
 // Attention kernels (seer_attn.cu).  Returns a cudaError_t.
 cudaError_t launch_attention(const AttnLaunch &p, cudaStream_t stream);
+// Block-sparse prefill with one head's query block per tile (seer_sparse.cu).
+cudaError_t launch_sparse_attention(const AttnLaunch &p, cudaStream_t stream);
 int attn_grid_size(int B, int Hq, int Hkv, int nb);
 
 // Gate kernels (seer_gate.cu).

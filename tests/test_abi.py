@@ -101,11 +101,27 @@ def test_gate_and_mask_argument_checks(L):
     assert L.seer_compact_mask(ctypes.byref(sh), None, p, p, None) == seer.SEER_ERR_INVALID_ARG
 
 
-def test_topk_counts_helper_matches_oracle(oracle):
-    for density in (0.1, 0.2, 0.3, 0.5, 1.0, 0.0):
-        got = seer.topk_counts(density, 300)
-        want = oracle.topk_counts(density, 300)
-        assert list(got) == list(want)
+@pytest.mark.parametrize("ff,fd", [(True, True), (True, False), (False, True), (False, False)])
+def test_topk_from_density_matches_oracle(oracle, ff, fd):
+    """The C library's per-row TopK counts equal the oracle's k_i rule for
+    densities across [0, 1] (including values whose products are exact
+    integers, where ceil is most fragile), above 1, and nb up to the maximum."""
+    densities = [0.0, 1e-6, 0.1, 0.17, 0.2, 0.25, 0.3, 1.0 / 3.0, 0.5, 0.7, 0.9, 0.999, 1.0, 1.5]
+    for nb in (1, 2, 33, 512, 16384):
+        for density in densities:
+            got = seer.seer_topk_from_density(density, nb, ff, fd)
+            if nb <= 512 or density in (0.1, 1.0 / 3.0, 1.0):
+                want = oracle.topk_counts(density, nb, force_first=ff, force_diag=fd)
+                assert got == list(want), (nb, density)
+            assert all(1 <= k <= i + 1 for i, k in enumerate(got)) or not (ff or fd)
+
+
+def test_topk_from_density_rejects_bad_arguments(L):
+    out = (ctypes.c_int32 * 4)(7, 7, 7, 7)
+    for density, nb in ((float("nan"), 4), (-0.5, 4), (float("inf"), 4), (0.5, 0), (0.5, 16385)):
+        assert L.seer_topk_from_density(ctypes.c_double(density), nb, 1, 1, out) == seer.SEER_ERR_INVALID_ARG
+    assert list(out) == [7, 7, 7, 7]
+    assert L.seer_topk_from_density(ctypes.c_double(0.5), 4, 1, 1, None) == seer.SEER_ERR_INVALID_ARG
 
 
 def test_ragged_sequence_accepted(L):

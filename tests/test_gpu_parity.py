@@ -126,6 +126,37 @@ def test_prefill_shapes(oracle, B, Hq, Hkv, S, d, p, ff, fd):
     run_prefill_case(oracle, x["q"], x["k"], x["v"], mask)
 
 
+@pytest.mark.parametrize("d", [128, 64])
+def test_prefill_odd_counts_and_single_block_rows(oracle, d):
+    """Rows whose active count is odd (the kernel ends them with a one-block
+    step), rows holding a single block (the diagonal alone, or block 0 alone
+    with no diagonal), and even counts, all in one layer."""
+    B, Hq, Hkv, nb = 1, 4, 2, 24
+    S = nb * BLOCK
+    w = syn.custom("odd", B, Hq, Hkv, S, d, number=91 + d)
+    x = syn.make_inputs(w)
+    rng = np.random.default_rng(5 + d)
+    mask = np.zeros((B, Hq, nb, nb), np.uint8)
+    for h in range(Hq):
+        for i in range(nb):
+            kind = (h + i) % 5
+            if kind == 0:
+                sel = [i]                                   # the diagonal alone
+            elif kind == 1:
+                sel = [0]                                   # block 0 alone (no diagonal for i > 0)
+            elif kind == 2:
+                sel = rng.choice(i + 1, size=min(i + 1, 3), replace=False)
+            elif kind == 3:
+                n_odd = (i + 1) if (i + 1) % 2 else i       # the largest odd count <= i + 1
+                sel = rng.choice(i + 1, size=n_odd, replace=False)
+            else:
+                sel = rng.choice(i + 1, size=min(i + 1, 2), replace=False)
+            mask[0, h, i, sel] = 1
+    counts = mask.sum(-1)
+    assert (counts % 2 == 1).sum() > nb and (counts == 1).sum() >= 2 * Hq
+    run_prefill_case(oracle, x["q"], x["k"], x["v"], torch.from_numpy(mask))
+
+
 @pytest.mark.parametrize("B,Hq,Hkv,S,d,p", [
     (1, 4, 2, 5 * BLOCK + 17, 128, 0.5),      # ragged last block, head pairs
     (2, 3, 1, 3 * BLOCK + 1, 64, 0.6),        # a one-token last block, leftover head

@@ -7,6 +7,8 @@ the step time.  These tests check that plumbing and the per-rank inputs.
 import os
 import socket
 
+import numpy as np
+
 import pytest
 import torch
 import torch.multiprocessing as mp
@@ -91,3 +93,72 @@ def test_tile_order_covers_every_query_block_once(g):
             assert h // g == kvh
             seen[key] = u
     assert len(seen) == B * Hq * nb
+
+
+def _split_worker(rank, world, port, q):
+    """One rank of the KV-head split: the oracle's gate, TopK mask and masked
+    attention on this rank's head slice of one layer, gathered on rank 0."""
+    os.environ.update({"MASTER_ADDR": "127.0.0.1", "MASTER_PORT": str(port), "RANK": str(rank),
+                       "WORLD_SIZE": str(world), "LOCAL_RANK": str(rank)})
+    import bench
+    import oracle
+    from long_context_prefill_attngate_b200 import partition
+    from long_context_prefill_attngate_b200 import synthetic as syn
+    import torch.distributed as dist
+    w, r, _ = bench.dist_setup(world)
+    try:
+        wl = syn.custom("split", 1, 4, 2, 256, 64, number=17, d_gate=64)
+        x = syn.make_inputs(wl)                      # every rank draws the same layer
+        xs = partition.slice_layer(x, wl.Hq, wl.Hkv, w, r)
+        bits = lambda t: syn.bf16_bits(t)
+        s = oracle.gate_scores(bits(xs["q"]), bits(xs["k"]), bits(xs["wq"]), bits(xs["wk"]), theta=wl.rope_theta)
+        m = oracle.block_mask(s.astype(np.float32), "topk", k_row=oracle.topk_counts(0.5, wl.nb))
+        o, lse = oracle.masked_attention(bits(xs["q"]), bits(xs["k"]), bits(xs["v"]), m)
+        parts = [None] * w
+        dist.all_gather_object(parts, (r, s, m, o, lse))
+        if r == 0:
+            parts.sort(key=lambda p: p[0])
+            # scores and mask are [B, H, nb, nb]; O and LSE come per (b, h, i) unit, head-major for B = 1
+            q.put(tuple(np.concatenate([p[i] for p in parts], axis=1 if i <= 2 else 0) for i in range(1, 5)))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_kv_head_split_reassembles_single_rank_layer():
+    """World size 2 on CPU: each rank computes its KV-head group's slice of a
+    layer with the oracle; the slices, concatenated along the head axis, equal
+    the single-rank result bit for bit (scores, mask, O and LSE)."""
+    import oracle
+    from long_context_prefill_attngate_b200 import synthetic as syn
+    world = 2
+    ctx = mp.get_context("spawn")
+    qu = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_split_worker, args=(r, world, port, qu)) for r in range(world)]
+    for p in procs:
+        p.start()
+    got = qu.get(timeout=300)
+    for p in procs:
+        p.join(timeout=120)
+        assert p.exitcode == 0
+    wl = syn.custom("split", 1, 4, 2, 256, 64, number=17, d_gate=64)
+    x = syn.make_inputs(wl)
+    bits = lambda t: syn.bf16_bits(t)
+    s = oracle.gate_scores(bits(x["q"]), bits(x["k"]), bits(x["wq"]), bits(x["wk"]), theta=wl.rope_theta)
+    m = oracle.block_mask(s.astype(np.float32), "topk", k_row=oracle.topk_counts(0.5, wl.nb))
+    o, lse = oracle.masked_attention(bits(x["q"]), bits(x["k"]), bits(x["v"]), m)
+    for a, b in zip(got, (s, m, o, lse)):
+        assert a.shape == b.shape
+        assert np.array_equal(a, b)
+
+
+def test_head_range_partition():
+    from long_context_prefill_attngate_b200 import partition
+    assert partition.head_range(32, 8, 4, 1) == (8, 16, 2, 4)
+    assert partition.head_range(40, 8, 8, 7) == (35, 40, 7, 8)
+    spans = [partition.head_range(32, 8, 2, r) for r in range(2)]
+    assert spans == [(0, 16, 0, 4), (16, 32, 4, 8)]
+    with pytest.raises(ValueError):
+        partition.head_range(32, 8, 3, 0)
+    with pytest.raises(ValueError):
+        partition.head_range(32, 8, 2, 2)
