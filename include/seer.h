@@ -188,12 +188,14 @@ SEER_API seer_status seer_compact_mask(const seer_shape *shape, const uint8_t *m
  * softmax_scale <= 0 selects 1/sqrt(d).  q, k, v, o must be 16-B aligned.
  * Workspace: seer_workspace_bytes(SEER_CALL_BLOCK_SPARSE_PREFILL) (may be 0;
  * workspace may then be NULL).
- * Scheduling: the persistent grid's tile slots take tiles from a counter
- * that the call zeroes on `stream` (an 8-byte memset before the launch);
- * counters come from a per-device ring of 256, so up to 256 prefill / pooled-
- * map launches may be in flight at once on any streams.  A CUDA graph that
- * captured the call reuses its counter on every replay, so one graph must
- * not be replayed on two streams at once.
+ * Scheduling: the persistent grid takes tiles from a counter that the call
+ * seeds on `stream` (an 8-byte memset before the launch); counters come from
+ * a per-device ring of 256, so up to 256 prefill / pooled-map launches may be
+ * in flight at once on any streams.  A launch whose counter slot is re-seeded
+ * by a later launch while it still runs stops taking tiles and records a
+ * device error that seer_check_status reports as SEER_ERR_DEVICE.  A CUDA
+ * graph that captured the call reuses its counter on every replay, so one
+ * graph must not be replayed on two streams at once.
  */
 SEER_API seer_status seer_block_sparse_prefill(const seer_shape *shape, const void *q, const void *k,
                                       const void *v, const uint8_t *mask, float softmax_scale,
@@ -223,9 +225,13 @@ SEER_API seer_status seer_attn_pooled_map(const seer_shape *shape, const void *q
  * pages have no counterpart; it is a deployment convenience.  Same inputs,
  * outputs and results as seer_gate_scores, but the workspace comes from a
  * fixed 24 MiB device array inside the library (held by every GPU that loads
- * the library until exit).  Shapes whose gate workspace
- * (seer_workspace_bytes(SEER_CALL_GATE_SCORES) for the given d_gate) exceeds
- * 24 MiB return SEER_ERR_UNSUPPORTED and launch nothing.  The first call on a
+ * the library until exit).  The gate needs, with nb = ceil(S/64),
+ * dk = d (average K pooling) or 2d (max+min) and each term rounded up to a
+ * multiple of 256 bytes,
+ *   4 B*Hq*nb*d + 4 B*Hkv*nb*dk + 4 B*Hq*nb*d_gate + 4 B*Hkv*nb*d_gate  bytes;
+ * shapes for which that exceeds 24 MiB (25165824 bytes) return
+ * SEER_ERR_UNSUPPORTED and launch nothing.  (seer_workspace_bytes reports a
+ * d_gate = 256, max+min bound and is not this call's limit.)  The first call on a
  * device looks up the array's device address; make it before any stream
  * capture.  All calls share the array: calls whose kernels overlap on the GPU
  * race and must be ordered (one stream, or events).

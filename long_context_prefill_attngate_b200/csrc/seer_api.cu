@@ -22,8 +22,9 @@ namespace seer {
 __device__ int g_status_word;
 
 // Tile counters of the attention launches: a ring per device, one slot per
-// launch, zeroed on the launch stream.  256 launches can be in flight at once
-// (on any number of streams) before a slot is reused.
+// launch, seeded on the launch stream.  256 launches can be in flight at once
+// (on any number of streams) before a slot is reused; a kernel that finds its
+// slot re-seeded by a later launch records kStatusRing (SEER_ERR_DEVICE).
 constexpr int kTileCounterRing = 256;
 __device__ unsigned long long g_tile_counters[kTileCounterRing];
 
@@ -93,8 +94,9 @@ int *status_ptr()
 }
 
 // A tile counter for one attention launch: the next slot of this device's
-// ring, zeroed on `stream` before the launch.  Null on a CUDA error (in *err).
-unsigned long long *tile_counter(cudaStream_t stream, cudaError_t *err)
+// ring, seeded on `stream` before the launch with a byte pattern (*base) that
+// changes every time the slot comes round again.  Null on a CUDA error (in *err).
+unsigned long long *tile_counter(cudaStream_t stream, cudaError_t *err, unsigned long long *base)
 {
     static std::mutex mu;
     static unsigned long long *cache[64] = {nullptr};
@@ -108,6 +110,7 @@ unsigned long long *tile_counter(cudaStream_t stream, cudaError_t *err)
         return nullptr;
     }
     unsigned long long *c = nullptr;
+    int tag = 1;
     {
         std::lock_guard<std::mutex> lk(mu);
         if (cache[dev] == nullptr) {
@@ -117,9 +120,12 @@ unsigned long long *tile_counter(cudaStream_t stream, cudaError_t *err)
                 return nullptr;
             cache[dev] = static_cast<unsigned long long *>(ptr);
         }
-        c = cache[dev] + (next[dev]++ % kTileCounterRing);
+        const unsigned seq = next[dev]++;
+        c = cache[dev] + (seq % kTileCounterRing);
+        tag = (int)((seq / kTileCounterRing) % 255u) + 1;
     }
-    *err = cudaMemsetAsync(c, 0, sizeof(unsigned long long), stream);
+    *base = 0x0101010101010101ull * (unsigned long long)tag;
+    *err = cudaMemsetAsync(c, tag, sizeof(unsigned long long), stream);
     return *err == cudaSuccess ? c : nullptr;
 }
 
@@ -371,7 +377,7 @@ seer_status seer_block_sparse_prefill(const seer_shape *shape, const void *q, co
     a.timeout_ns = g_timeout_ns;
     a.status = status;
     cudaError_t e = cudaSuccess;
-    a.tile_ctr = tile_counter(static_cast<cudaStream_t>(stream), &e);
+    a.tile_ctr = tile_counter(static_cast<cudaStream_t>(stream), &e, &a.tile_base);
     if (a.tile_ctr == nullptr)
         return cuda_fail(e, "seer_block_sparse_prefill tile counter");
     e = launch_attention(a, static_cast<cudaStream_t>(stream));
@@ -421,7 +427,7 @@ seer_status seer_attn_pooled_map(const seer_shape *shape, const void *q, const v
     a.map_mode = true;
     a.timeout_ns = g_timeout_ns;
     a.status = status;
-    a.tile_ctr = tile_counter(s, &e);
+    a.tile_ctr = tile_counter(s, &e, &a.tile_base);
     if (a.tile_ctr == nullptr)
         return cuda_fail(e, "seer_attn_pooled_map tile counter");
     e = launch_attention(a, s);
@@ -459,6 +465,9 @@ seer_status seer_check_status(void *stream)
         cudaMemcpyToSymbol(g_status_word, &zero, sizeof(int));
         if (v == kStatusTimeout)
             return fail(SEER_ERR_TIMEOUT, "a device-side wait ran out");
+        if (v == kStatusRing)
+            return fail(SEER_ERR_DEVICE, "more than 256 attention launches were in flight at once: a tile-counter "
+                                         "slot was reused by a later launch (outputs of the earlier one are incomplete)");
         return fail(SEER_ERR_DEVICE, "device-side check failed (code %d)", v);
     }
     return ok();

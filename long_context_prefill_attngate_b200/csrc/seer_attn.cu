@@ -73,7 +73,8 @@ struct KParams {
     int *status;
     int nslots;              // independent tiles in flight per CTA (1 or 2)
     int slot_bytes;          // shared memory per slot
-    unsigned long long *tile_ctr;   // next tile of the launch (zeroed before it)
+    unsigned long long *tile_ctr;   // next tile of the launch (seeded with tile_base before it)
+    unsigned long long tile_base;
 };
 
 // Tile order: KV-head major, so the CTAs running at any moment read the K/V
@@ -255,9 +256,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         while (true) {
             long long u = 0;
             if (lane == 0)
-                u = (long long)atomicAdd(p.tile_ctr, 1ull);
+                u = next_tile(p.tile_ctr, p.tile_base, p.status);
             u = __shfl_sync(0xffffffffu, u, 0);
-            const bool end = u >= p.n_units;
+            const bool end = u < 0 || u >= p.n_units;
             Unit un{};
             if (!end) {
                 un = decode_unit(p, u);
@@ -739,6 +740,7 @@ cudaError_t launch_t(const AttnLaunch &a, cudaStream_t stream)
     p.timeout_ns = a.timeout_ns;
     p.status = a.status;
     p.tile_ctr = a.tile_ctr;
+    p.tile_base = a.tile_base;
     // Two tile slots per CTA when their shared memory fits (227 KB per CTA).
     p.nslots = Smem<D>::total_bytes(a.nb, 2) <= 227 * 1024 ? 2 : 1;
     p.slot_bytes = Smem<D>::slot_bytes(a.nb);

@@ -31,7 +31,8 @@ struct AttnLaunch {
     bool map_mode;
     uint64_t timeout_ns;
     int *status;                  // device status word
-    unsigned long long *tile_ctr; // tile counter of this launch, zeroed on the launch stream
+    unsigned long long *tile_ctr; // tile counter of this launch, seeded with tile_base on the launch stream
+    unsigned long long tile_base;
 };
 
 // Attention kernels (seer_attn.cu).  Returns a cudaError_t.

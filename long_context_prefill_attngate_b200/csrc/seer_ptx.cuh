@@ -10,12 +10,27 @@ namespace seer {
 
 // Device status codes written through the status pointer every kernel gets
 // (first error wins).
-enum : int { kStatusOk = 0, kStatusTimeout = 5, kStatusDevice = 6 };
+enum : int { kStatusOk = 0, kStatusTimeout = 5, kStatusDevice = 6, kStatusRing = 7 };
 
 __device__ __forceinline__ void set_status(int *status, int s)
 {
     if (status != nullptr)
         atomicCAS(status, 0, s);
+}
+
+// Next tile of a launch from its counter slot.  The host seeds the slot with
+// `base`, a byte pattern that differs between successive users of the slot;
+// a value far from it means a later launch re-seeded the slot while this one
+// was still taking tiles (more launches in flight than the ring has slots):
+// the status word records kStatusRing and -1 (no more tiles) is returned.
+__device__ __forceinline__ long long next_tile(unsigned long long *ctr, unsigned long long base, int *status)
+{
+    const unsigned long long u = atomicAdd(ctr, 1ull) - base;
+    if (u >= (1ull << 40)) {
+        set_status(status, kStatusRing);
+        return -1;
+    }
+    return (long long)u;
 }
 
 __device__ __forceinline__ uint32_t smem_u32(const void *p)

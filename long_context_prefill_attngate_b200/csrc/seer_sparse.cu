@@ -14,16 +14,18 @@
 //    instead: each step takes TWO selected key blocks, S = Q K^T with N = 128
 //    (and O += P V with K = 128 keys, N = d).  A row with an odd count ends with
 //    a single-block step (N = 64, K = 64), so nothing is padded.
-//  * TMEM: one S (128 fp32 columns), three P buffers (64 columns of packed
-//    bf16 each; PV reads P from TMEM as a TS MMA) and one O (128).  S is free
-//    again as soon as the softmax has loaded it, early in the step, so S(t + 1)
-//    runs while the softmax of t computes.  P(t) is written into buffer t % 3;
-//    the S issuer starts S(t) only once PV(t - 3) has completed, so the
-//    softmax, having seen S(t), never waits for a P buffer.  M = 64 rows live in lanes
+//  * TMEM: three S buffers (128 fp32 columns each) and one O (128).  P(t)
+//    (packed bf16) overwrites the first 64 columns of S buffer t % 3 and PV
+//    reads it from there as a TS MMA.  S(t) is issued once PV(t - 3) has
+//    completed, so S runs two steps ahead of the softmax and the tensor pipe
+//    never waits for the softmax's reads; the softmax waits only for S(t).
+//    M = 64 rows live in lanes
 //    32 (m / 16) + m % 16.  Eight softmax warps, two per lane quarter: both
 //    load the row's whole S (the 16x32bx2 shape: thread c holds key block c),
 //    so each has the exact row max without exchanging it, and they split the
 //    exponentials (keys 0-31 / 32-63 of each block) and the output's d columns.
+//    The pair meets at one barrier per step before P overwrites the S they
+//    both read.
 //  * Two MMA-issuing threads: one issues the S MMAs, the other the PV MMAs.
 //    A tcgen05.mma issue blocks at the tensor pipe's rate and every commit or
 //    barrier check of the issuing thread is serial latency; with two issuers
@@ -77,6 +79,7 @@ struct SParams {
     uint64_t timeout_ns;
     int *status;
     unsigned long long *tile_ctr;
+    unsigned long long tile_base;
     int list_stride;
 };
 
@@ -90,10 +93,11 @@ struct Geo {
     static constexpr int kOffV = kOffK + 2 * kStage;
     static constexpr int kOffBar = kOffV + 2 * kStage;
     // barriers, two of each (indexed by buffer / stage / step parity)
-    // s_full / s_free / p_full alternate by step parity, pv_done cycles over the three P buffers.
-    static constexpr int kQFull = 0, kQEmpty = 2, kKFull = 4, kVFull = 6, kSFull = 8, kSFree = 10, kPFull = 12,
-                         kPVDone = 14, kOFull = 17, kOFree = 19, kListFull = 21, kListEmpty = 23, kDrain = 25,
-                         kNumBars = 27;
+    // s_full, p_full and pv_done cycle over the three S buffers (step % 3): S may
+    // run two steps ahead of the softmax, and three slots keep every parity wait
+    // unambiguous (S(t + 3) cannot complete before the softmax has read S(t)).
+    static constexpr int kQFull = 0, kQEmpty = 2, kKFull = 4, kVFull = 6, kSFull = 8, kPFull = 11, kPVDone = 14,
+                         kOFull = 17, kOFree = 19, kListFull = 21, kListEmpty = 23, kDrain = 25, kNumBars = 27;
     static constexpr int kOffXch = kOffBar + kNumBars * 8;         // float [2 slots][4 quarters][2 halves][16 rows]
     static constexpr int kOffInfo = kOffXch + 2 * 4 * 2 * 16 * 4;
     static constexpr int kOffMisc = kOffInfo + 2 * (int)sizeof(TileInfo);
@@ -108,9 +112,20 @@ __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, const W
     return __all_sync(0xffffffffu, r);
 }
 
-__device__ __forceinline__ void named_bar_arrive(int id, int nthreads)
+// Barrier of the two softmax warps that share a lane quarter (64 threads).  The
+// non-aligned forms are used: they stay correct even if a warp reaches them
+// before it has reconverged, and the arrive-only form releases a waiting
+// partner when a warp leaves on an abort.
+__device__ __forceinline__ void pair_bar_sync(int id)
 {
-    asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+    __syncwarp();
+    asm volatile("barrier.sync %0, 64;" ::"r"(id) : "memory");
+}
+
+__device__ __forceinline__ void pair_bar_arrive(int id)
+{
+    __syncwarp();
+    asm volatile("barrier.arrive %0, 64;" ::"r"(id) : "memory");
 }
 
 template <int D>
@@ -143,7 +158,6 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(bar(G::kKFull + x), 1);
             mbar_init(bar(G::kVFull + x), 1);
             mbar_init(bar(G::kSFull + x), 1);
-            mbar_init(bar(G::kSFree + x), kSoftmaxWarps);
             mbar_init(bar(G::kPFull + x), kSoftmaxWarps);
             mbar_init(bar(G::kPVDone + x), 1);
             mbar_init(bar(G::kOFull + x), 1);
@@ -152,6 +166,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(bar(G::kListEmpty + x), kListConsumers);
             mbar_init(bar(G::kDrain + x), 1);
         }
+        mbar_init(bar(G::kSFull + 2), 1);
+        mbar_init(bar(G::kPFull + 2), kSoftmaxWarps);
         mbar_init(bar(G::kPVDone + 2), 1);
         *abort_flag = 0;
         fence_mbar_init();
@@ -169,9 +185,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_base_ptr;
-    const uint32_t tS = tmem;
-    auto tP = [&](int b) -> uint32_t { return tmem + 128u + 64u * (uint32_t)b; };
-    const uint32_t tO = tmem + 320u;
+    auto tS = [&](int b) -> uint32_t { return tmem + 128u * (uint32_t)b; };   // b = step % 3; P aliases it
+    const uint32_t tO = tmem + 384u;
 
     if (warp == kWarpList) {
         // ------------------------------------------------------------ list builder
@@ -180,12 +195,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         while (true) {
             long long u = 0;
             if (lane == 0)
-                u = (long long)atomicAdd(p.tile_ctr, 1ull);
+                u = next_tile(p.tile_ctr, p.tile_base, p.status);
             u = __shfl_sync(0xffffffffu, u, 0);
             const int lb = n & 1;
             if (n >= 2 && !warp_wait(bar(G::kListEmpty + lb), ((n >> 1) - 1) & 1, wc))
                 break;
-            if (u >= p.n_units) {
+            if (u < 0 || u >= p.n_units) {
                 if (lane == 0) {
                     infos[lb].count = -1;
                     mbar_arrive(bar(G::kListFull + lb));
@@ -239,7 +254,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else if (warp == kWarpQK || warp == kWarpV) {
         // ------------------------------------------------------------ TMA producers
         // Stage s of step t is free once the MMA of step t - 2 has completed:
-        // S (the K ring) commits to s_full[t & 1], PV (the V ring) to pv_done[t % 3].
+        // S (the K ring) commits to s_full[t % 3], PV (the V ring) to pv_done[t % 3].
         const bool kprod = warp == kWarpQK;
         if (lane == 0) {
             int n = 0, q_it = 0, it = 0;
@@ -275,8 +290,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                     for (int s = 0; s < steps; ++s) {
                         const int st = it & 1;
                         const bool freed =
-                            it < 2 || (kprod ? mbar_wait(bar(G::kSFull + st), (uint32_t)(((it >> 1) - 1) & 1), wc)
-                                             : mbar_wait(bar(G::kPVDone + (it - 2) % 3), (uint32_t)(((it - 2) / 3) & 1), wc));
+                            it < 2 || mbar_wait(bar((kprod ? G::kSFull : G::kPVDone) + (it - 2) % 3),
+                                                (uint32_t)(((it - 2) / 3) & 1), wc);
                         if (!freed) {
                             ok = false;
                             break;
@@ -364,10 +379,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int steps = (count + 1) >> 1;
                 for (int s = 0; s < steps; ++s, ++g) {
                     const int sb = g & 1;
-                    // K of this step landed; S free (the softmax has loaded S(g - 1)); P
-                    // buffer g % 3 free (PV(g - 3) completed) before the softmax sees S(g).
+                    // K of this step landed; S buffer g % 3 free: PV(g - 3) has read the P
+                    // written over it (and so the softmax has read S(g - 3)).
                     if (!mbar_wait(bar(G::kKFull + sb), (uint32_t)((g >> 1) & 1), wc) ||
-                        (g >= 1 && !mbar_wait(bar(G::kSFree + (sb ^ 1)), (uint32_t)(((g - 1) >> 1) & 1), wc)) ||
                         (g >= 3 && !mbar_wait(bar(G::kPVDone + g % 3), (uint32_t)(((g - 3) / 3) & 1), wc))) {
                         ok = false;
                         break;
@@ -379,10 +393,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                     for (int kk = 0; kk < D / 16; ++kk) {
                         const uint32_t qo = ((kk >> 2) * 8192 + (kk & 3) * 32) >> 4;
                         const uint32_t ko = ((kk >> 2) * 16384 + (kk & 3) * 32) >> 4;
-                        mma_ss(tS, dq + qo, dk + ko, id, kk > 0 ? 1u : 0u);
+                        mma_ss(tS(g % 3), dq + qo, dk + ko, id, kk > 0 ? 1u : 0u);
                     }
                     issued = true;
-                    tc_commit(bar(G::kSFull + sb));
+                    tc_commit(bar(G::kSFull + g % 3));
                     if (s == steps - 1)
                         tc_commit(bar(G::kQEmpty + qb));
                 }
@@ -420,7 +434,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const int sb = g & 1;
                     // The first PV of a tile overwrites O: the previous tile's O must
                     // have been read out (o_free).
-                    if (!mbar_wait(bar(G::kPFull + sb), (uint32_t)((g >> 1) & 1), wc) ||
+                    if (!mbar_wait(bar(G::kPFull + g % 3), (uint32_t)((g / 3) & 1), wc) ||
                         !mbar_wait(bar(G::kVFull + sb), (uint32_t)((g >> 1) & 1), wc) ||
                         (s == 0 && o_it >= 1 && !mbar_wait(bar(G::kOFree + (o_it - 1) % 2), (uint32_t)(((o_it - 1) >> 1) & 1), wc))) {
                         ok = false;
@@ -432,7 +446,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     for (int kk = 0; kk < ksteps; ++kk) {
                         // V stage [block][panel][64 keys]: 16 keys per K step, LBO = next d panel.
                         const uint32_t vo = ((kk >> 2) * G::kBlkBytes + (kk & 3) * 2048) >> 4;
-                        mma_ts(tO, tP(g % 3) + kk * 8, dv + vo, idPV, (s == 0 && kk == 0) ? 0u : 1u);
+                        mma_ts(tO, tS(g % 3) + kk * 8, dv + vo, idPV, (s == 0 && kk == 0) ? 0u : 1u);
                     }
                     issued = true;
                     tc_commit(bar(G::kPVDone + g % 3));
@@ -467,7 +481,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             float *xs = xch + (xcnt & 1) * 128 + qt * 32;
             if (lane < 16)
                 xs[hf * 16 + lane] = val;
-            named_bar_sync(pair_bar, 64);
+            pair_bar_sync(pair_bar);
             const float o = xs[(hf ^ 1) * 16 + (lane & 15)];
             ++xcnt;
             return o;
@@ -548,21 +562,17 @@ __global__ void __launch_bounds__(kThreads, 1)
             // instantiation so the other steps carry no masking code.
             auto step = [&](auto last_c) -> bool {
                 constexpr bool kLast = decltype(last_c)::value;
-                if (!warp_wait(bar(G::kSFull + (g & 1)), (uint32_t)((g >> 1) & 1), wc))
+                if (!warp_wait(bar(G::kSFull + g % 3), (uint32_t)((g / 3) & 1), wc))
                     return false;
                 tc_fence_after();
                 // Thread c holds key block c: v = this warp's 32 keys (32 hf ..), w = the
                 // other warp's 32 (only their max is needed).
                 const int e = 2 * s + c;              // list entry of this thread's key block
+                const uint32_t tSg = tS(g % 3);
                 uint32_t v[32], w[32];
-                tmem_ld16x2_32<64>(tS + lane_off + hf * 32, v);
-                tmem_ld16x2_32<64>(tS + lane_off + (hf ^ 1) * 32, w);
+                tmem_ld16x2_32<64>(tSg + lane_off + hf * 32, v);
+                tmem_ld16x2_32<64>(tSg + lane_off + (hf ^ 1) * 32, w);
                 tmem_wait_ld();
-                // S(g) is in registers: S may take S(g + 1).
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0)
-                    mbar_arrive(bar(G::kSFree + (g & 1)));
                 if constexpr (kLast) {
                     // Keys kept in each half: none for an absent block; up to the query
                     // row in the diagonal block (causal); all otherwise.
@@ -639,14 +649,17 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                 }
                 l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
-                // Keys 32 hf + 2k, +1 of block c in P column 32 c + 16 hf + k.  (P buffer
-                // g % 3 is free: S(g) was only issued after PV(g - 3) completed.)
-                tmem_st16x2_16<32>(tP(g % 3) + lane_off + hf * 16, pk);
+                // Both warps of the pair have loaded S(g): P may overwrite it.  Keys
+                // 32 hf + 2k, +1 of block c go to column 32 c + 16 hf + k.
+                tc_fence_before();
+                pair_bar_sync(pair_bar);
+                tc_fence_after();
+                tmem_st16x2_16<32>(tSg + lane_off + hf * 16, pk);
                 tmem_wait_st();
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0)
-                    mbar_arrive(bar(G::kPFull + (g & 1)));
+                    mbar_arrive(bar(G::kPFull + g % 3));
                 // The previous tile's O: its last PV finished while this step ran;
                 // this tile's first PV waits for it to be read out.
                 if (pend && !epilogue())
@@ -676,10 +689,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (ok && pend)
             epilogue();
         if (!ok) {
-            // The partner warp may be waiting in a pair exchange (at most two come
+            // The partner warp may be waiting at a pair barrier (at most two come
             // between bounded waits, which see the abort flag): release it.
-            named_bar_arrive(pair_bar, 64);
-            named_bar_arrive(pair_bar, 64);
+            pair_bar_arrive(pair_bar);
+            pair_bar_arrive(pair_bar);
         }
     }
 
@@ -714,6 +727,7 @@ cudaError_t launch_d(const AttnLaunch &a, cudaStream_t stream)
     p.timeout_ns = a.timeout_ns;
     p.status = a.status;
     p.tile_ctr = a.tile_ctr;
+    p.tile_base = a.tile_base;
     p.list_stride = Geo<D>::list_stride(a.nb);
     const int smem = Geo<D>::smem_bytes(a.nb);
     if (smem > 227 * 1024)

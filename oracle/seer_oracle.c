@@ -14,10 +14,10 @@
  *  [GATE]  "SeerAttention: Learning Intrinsic Sparse Attention in Your LLMs",
  *          rebuttal, Weakness 3 (pooling along the sequence axis, shapes
  *          [Batch, Head, Seq/Block, Dim], pooling before the linear layer),
- *          Question 1 on pooling ("Q prefers avg"), Q1 on AttnGate's RoPE
- *          (block RoPE on non-RoPE'd pooled Q/K), Weakness 2 (the gate is
- *          "similar to self-attention without the multiply with V"; per-row
- *          TopK; [Seq/Block, TopK] index tensor).
+ *          Question 1 on pooling (average pooling suits Q), Q1 on AttnGate's
+ *          RoPE (block RoPE on non-RoPE'd pooled Q/K), Weakness 2 (the gate
+ *          is an attention score computation that stops before the product
+ *          with V; per-row TopK; [Seq/Block, TopK] index tensor).
  *  [CARD]  "SeerAttention-Llama-3.1-8B-AttnGates" model card: masks come from
  *          threshold/TopK on the gate's soft scores and drive a block-sparse
  *          FlashAttention kernel.
@@ -95,9 +95,9 @@ void oracle_pool_avg(const uint16_t *x, int B, int H, int S, int d, double *out)
 }
 
 /* ---------------------------------------------------------------------------
- * a1' [GATE Weakness 3: "Max+Min pooling in K ... concated in hidden dim
- * before the linear layer ([Batch, Head, Seq / Block, Dim * 2])"; Question 1:
- * K prefers max-min pooling]:
+ * a1' [GATE Weakness 3: K may be pooled by per-block max and min, the two
+ * results joined along the feature axis (2 d features per block) ahead of
+ * the linear layer; Question 1: max-min pooling suits K]:
  * out[b,h,i,c]     = max_{t<n_i} x[b,h,64 i + t, c]
  * out[b,h,i,d + c] = min_{t<n_i} x[b,h,64 i + t, c]      (max first: a reading)
  * x: bf16 [B, H, S, d]  ->  out: f64 [B, H, nb, 2d]
@@ -172,8 +172,9 @@ void oracle_project_rope(const double *xp, int B, int H, int nb, int d,
 }
 
 /* ---------------------------------------------------------------------------
- * a3 [GATE Weakness 2: "similar to self-attention without the multiply with
- * V"; Question 2: the gate output rows sum to 1]:
+ * a3 [GATE Weakness 2: the gate scores blocks the way attention scores
+ * tokens, without the product with V; Question 2: the gate output rows sum
+ * to 1]:
  * G[b,h,i,j] = softmax_{j<=i}( qt[b,h,i] . kt[b,h/g,j] / sqrt(dg) ), 0 for j>i.
  * Full chain: pool Q and K, project + block RoPE, causal block softmax.
  * scores: f64 [B, Hq, nb, nb].
@@ -319,7 +320,7 @@ void oracle_block_mask(const float *scores, int B, int Hq, int nb, int mode,
 }
 
 /* ---------------------------------------------------------------------------
- * a5 [INF: "for j from 1 to TopK ... sparse block index"; GATE Weakness 2:
+ * a5 [INF: the kernel loops over the row's TopK selected block indices; GATE Weakness 2:
  * [Seq/Block, TopK] index tensor]: per (b, h, i) the ascending list of active
  * key blocks j <= i.  Lists are stored causal-packed: row i of head (b, h)
  * starts at (b*Hq + h) * nb(nb+1)/2 + i(i+1)/2 and has room for i+1 entries;

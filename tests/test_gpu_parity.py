@@ -445,18 +445,30 @@ def test_llama8k_threshold_layer(oracle):
     run_prefill_case(oracle, x["q"], x["k"], x["v"], m.cpu(), units=sample_units(1, w.Hq, w.nb, 4, 1))
 
 
-def test_llama32k_topk_layer(oracle):
-    """The benchmark's launch configuration: 32k, TopK density 0.1."""
+@pytest.fixture(scope="module")
+def llama32k(oracle):
     w = syn.WORKLOADS["llama8b_32k"]
     x = syn.make_inputs(w)
-    s, m = _gate_mask(w, x, "topk", density=0.1)
-    k_row = oracle.topk_counts(0.1, w.nb)
+    ref_rows = oracle.gate_scores(bits(x["q"]), bits(x["k"]), bits(x["wq"]), bits(x["wk"]), theta=w.rope_theta)
+    return w, x, ref_rows
+
+
+@pytest.mark.parametrize("density", [1.0, 0.5, 0.3, 0.2, 0.1])
+def test_llama32k_topk_layer(oracle, llama32k, density):
+    """The benchmark's launch configuration: 32k, every TopK density of the
+    sweep (1.0 is the dense causal point).  Scores within rel 1e-2, the mask
+    bit-exact, O on sampled query blocks of every head."""
+    w, x, ref_rows = llama32k
+    s, m = _gate_mask(w, x, "topk", density=density)
+    k_row = oracle.topk_counts(density, w.nb)
     sc = s.cpu().numpy()
     ref_m = oracle.block_mask(sc, "topk", k_row=k_row)
     assert np.array_equal(m.cpu().numpy(), ref_m)
-    ref_rows = oracle.gate_scores(bits(x["q"]), bits(x["k"]), bits(x["wq"]), bits(x["wk"]), theta=w.rope_theta)
     check_rel(sc, ref_rows, "scores@32k")
-    run_prefill_case(oracle, x["q"], x["k"], x["v"], m.cpu(), units=sample_units(1, w.Hq, w.nb, 4, 2))
+    del sc, ref_m
+    n_blocks = 3 if density >= 0.5 else 4
+    run_prefill_case(oracle, x["q"], x["k"], x["v"], m.cpu(),
+                     units=sample_units(1, w.Hq, w.nb, n_blocks, 2 + int(density * 10)))
 
 
 def test_llama128k_threshold_layer(oracle):
