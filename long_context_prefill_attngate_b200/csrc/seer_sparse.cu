@@ -17,34 +17,38 @@
 //  * TMEM: three S buffers (128 fp32 columns each) and one O (128).  P(t)
 //    (packed bf16) overwrites the first 64 columns of S buffer t % 3 and PV
 //    reads it from there as a TS MMA.  S(t) is issued once PV(t - 3) has
-//    completed, so S runs two steps ahead of the softmax and the tensor pipe
-//    never waits for the softmax's reads; the softmax waits only for S(t).
-//    M = 64 rows live in lanes
-//    32 (m / 16) + m % 16.  Eight softmax warps, two per lane quarter: both
-//    load the row's whole S (the 16x32bx2 shape: thread c holds key block c),
-//    so each has the exact row max without exchanging it, and they split the
-//    exponentials (keys 0-31 / 32-63 of each block) and the output's d columns.
-//    The pair meets at one barrier per step before P overwrites the S they
-//    both read.
+//    completed, so S runs two steps ahead of the softmax: the softmax of a step
+//    has about two steps of tensor-pipe time before its P is needed.  M = 64
+//    rows live in lanes 32 (m / 16) + m % 16.
+//  * Softmax: two groups of four warps take alternate steps (group = step % 2),
+//    one warp per TMEM lane quarter.  With the 16x32bx2 load shape thread c of a
+//    warp holds key block c of the step (64 scores in registers), so a row's
+//    max is one shuffle; the running max is handed from one group to the other
+//    through shared memory (one mbarrier per lane quarter).  The two groups'
+//    exponentials fall in different phases, so they share the SFU instead of
+//    colliding on it, and no warp waits for a partner within a step.  The
+//    running max moves only when it grows by more than 2^8 (log2 domain): P
+//    stays <= 256 and the O rescale (a TMEM round trip) is rare.  Each group
+//    keeps its own row sum, rescaled when it sees the max move; the two sums
+//    meet in the epilogue.
 //  * Two MMA-issuing threads: one issues the S MMAs, the other the PV MMAs.
 //    A tcgen05.mma issue blocks at the tensor pipe's rate and every commit or
 //    barrier check of the issuing thread is serial latency; with two issuers
 //    one thread's checks are covered by the other's MMAs.
-//  * K and V rings are two steps deep, so "stage free" is the same event as
-//    "S (or PV) of the step two back completed": one commit per step and issuer.
-//  * Warps: 0-7 softmax and epilogue (warp w = rows 16 (w % 4) .. + 15, key
-//    block / d half w / 4; a tile's O -> bf16 -> global and LSE are read out
-//    right after the softmax of the next tile's first step, and the next tile's
-//    first PV waits for that), 8 TMA for Q and K, 9 S issuer, 10 mask -> list
-//    builder, 11 TMA for V, 12 PV issuer.  One CTA per SM,
-//    persistent, tiles taken from a launch-wide atomic counter in
+//  * K and V rings of pair stages (two key blocks each); each MMA chain commits
+//    the release of the stage it read.  A TMA instruction holds its issuing
+//    thread for a long time and one thread's copies complete roughly one after
+//    another, so every box of a stage is issued by its own lane.
+//  * Warps: 0-7 softmax and epilogue (a tile's O -> bf16 -> global and LSE are
+//    read out by the group that takes the next step, right after its P store,
+//    and the next tile's first PV waits for that), 8 TMA for Q and K, 9 S
+//    issuer, 10 mask -> list builder, 11 TMA for V, 12 PV issuer.  One CTA per
+//    SM, persistent, tiles taken from a launch-wide atomic counter in
 //    KV-head-major order (concurrent tiles share one KV head's K/V in L2), the
 //    longest causal rows first.
-//  * K stage = one step's two key blocks, laid out [d panel][128 keys][128 B]
-//    so a single N = 128 descriptor spans both; V stage = [block][d panel][64
-//    keys][128 B] (MN-major B operand).  Q is double-buffered across tiles.
-//  * The running max moves only when it grows by more than 2^8 (log2 domain):
-//    P stays <= 256 and the O rescale (a TMEM round trip) is rare.
+//  * K stage laid out [d panel][128 keys][128 B] so a single N = 128 descriptor
+//    spans both blocks; V stage [block][d panel][64 keys][128 B] (MN-major B
+//    operand).  Q is double-buffered across tiles.
 //  * Every wait is bounded; a wait that runs out raises the device status word,
 //    the CTA drains its in-flight copies and MMAs, frees TMEM and exits.
 #include <cuda_bf16.h>
@@ -54,16 +58,23 @@
 #include "seer_internal.h"
 #include "seer_ptx.cuh"
 
+#ifndef SEER_NK
+#define SEER_NK 2
+#endif
+#ifndef SEER_NV
+#define SEER_NV 2
+#endif
+
 namespace seer {
 
 namespace {
 
 constexpr int kThreads = 416;         // 13 warps (four on one SM sub-partition: <= 128 registers)
-constexpr int kPrefetchAhead = 4;     // L2 prefetch distance in list entries
 constexpr uint64_t kDrain = 200000000ull;
-constexpr int kSoftmaxWarps = 8;
+constexpr int kGroupWarps = 4;        // softmax warps per group (one per lane quarter)
 constexpr int kListConsumers = 12;    // Q/K and V producers, S and PV issuers, 8 softmax warps
 constexpr int kWarpQK = 8, kWarpS = 9, kWarpList = 10, kWarpV = 11, kWarpPV = 12;
+constexpr int kStepBlocks = 2;        // key blocks per step
 
 struct TileInfo {
     int count, b, h, i, diag;
@@ -88,18 +99,25 @@ struct Geo {
     static constexpr int kPanels = D / 64;
     static constexpr int kQBytes = 64 * D * 2;        // one query block
     static constexpr int kBlkBytes = 64 * D * 2;      // one key block (K or V)
-    static constexpr int kStage = 2 * kBlkBytes;      // two key blocks
-    static constexpr int kOffK = 2 * kQBytes;
-    static constexpr int kOffV = kOffK + 2 * kStage;
-    static constexpr int kOffBar = kOffV + 2 * kStage;
-    // barriers, two of each (indexed by buffer / stage / step parity)
+    static constexpr int kPair = 2 * kBlkBytes;       // a stage: two key blocks
+    static constexpr int kNK = SEER_NK, kNV = SEER_NV; // ring depths in stages
+    static constexpr int kQBufs = 2;                  // query-block buffers
+    static constexpr int kOffK = kQBufs * kQBytes;
+    static constexpr int kOffV = kOffK + kNK * kPair;
+    static constexpr int kOffBar = kOffV + kNV * kPair;
     // s_full, p_full and pv_done cycle over the three S buffers (step % 3): S may
     // run two steps ahead of the softmax, and three slots keep every parity wait
-    // unambiguous (S(t + 3) cannot complete before the softmax has read S(t)).
-    static constexpr int kQFull = 0, kQEmpty = 2, kKFull = 4, kVFull = 6, kSFull = 8, kPFull = 11, kPVDone = 14,
-                         kOFull = 17, kOFree = 19, kListFull = 21, kListEmpty = 23, kDrain = 25, kNumBars = 27;
-    static constexpr int kOffXch = kOffBar + kNumBars * 8;         // float [2 slots][4 quarters][2 halves][16 rows]
-    static constexpr int kOffInfo = kOffXch + 2 * 4 * 2 * 16 * 4;
+    // unambiguous (S(t + 3) cannot complete before P(t) has been written).
+    // m_ready[slot][quarter] hands the running max from one softmax group to the
+    // other (slot = step % 2); l_ready[slot][quarter] collects both groups' row
+    // sums of a tile (slot = tile % 2).
+    static constexpr int kQFull = 0, kQEmpty = 2, kKFull = 4, kKEmpty = kKFull + kNK, kVFull = kKEmpty + kNK,
+                         kVEmpty = kVFull + kNV, kSFull = kVEmpty + kNV, kPFull = kSFull + 3, kPVDone = kPFull + 3,
+                         kOFull = kPVDone + 3, kOFree = kOFull + 2, kListFull = kOFree + 2, kListEmpty = kListFull + 2,
+                         kDrain = kListEmpty + 2, kMReady = kDrain + 2, kLReady = kMReady + 8, kNumBars = kLReady + 8;
+    static constexpr int kOffM = kOffBar + kNumBars * 8;           // float [2 slots][64 rows]
+    static constexpr int kOffL = kOffM + 2 * 64 * 4;               // float [2 slots][2 groups][2 (l, m)][64 rows]
+    static constexpr int kOffInfo = kOffL + 2 * 2 * 2 * 64 * 4;
     static constexpr int kOffMisc = kOffInfo + 2 * (int)sizeof(TileInfo);
     static constexpr int kOffList = (kOffMisc + 16 + 15) / 16 * 16;
     static int list_stride(int nb) { return (nb + 7) / 8 * 8; }    // uint16 entries per buffer
@@ -110,22 +128,6 @@ __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, const W
 {
     const bool r = mbar_wait(bar, parity, w);
     return __all_sync(0xffffffffu, r);
-}
-
-// Barrier of the two softmax warps that share a lane quarter (64 threads).  The
-// non-aligned forms are used: they stay correct even if a warp reaches them
-// before it has reconverged, and the arrive-only form releases a waiting
-// partner when a warp leaves on an abort.
-__device__ __forceinline__ void pair_bar_sync(int id)
-{
-    __syncwarp();
-    asm volatile("barrier.sync %0, 64;" ::"r"(id) : "memory");
-}
-
-__device__ __forceinline__ void pair_bar_arrive(int id)
-{
-    __syncwarp();
-    asm volatile("barrier.arrive %0, 64;" ::"r"(id) : "memory");
 }
 
 template <int D>
@@ -155,20 +157,29 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int x = 0; x < 2; ++x) {
             mbar_init(bar(G::kQFull + x), 1);
             mbar_init(bar(G::kQEmpty + x), 1);
-            mbar_init(bar(G::kKFull + x), 1);
-            mbar_init(bar(G::kVFull + x), 1);
-            mbar_init(bar(G::kSFull + x), 1);
-            mbar_init(bar(G::kPFull + x), kSoftmaxWarps);
-            mbar_init(bar(G::kPVDone + x), 1);
             mbar_init(bar(G::kOFull + x), 1);
-            mbar_init(bar(G::kOFree + x), kSoftmaxWarps);
+            mbar_init(bar(G::kOFree + x), kGroupWarps);
             mbar_init(bar(G::kListFull + x), 1);
             mbar_init(bar(G::kListEmpty + x), kListConsumers);
             mbar_init(bar(G::kDrain + x), 1);
         }
-        mbar_init(bar(G::kSFull + 2), 1);
-        mbar_init(bar(G::kPFull + 2), kSoftmaxWarps);
-        mbar_init(bar(G::kPVDone + 2), 1);
+        for (int x = 0; x < G::kNK; ++x) {
+            mbar_init(bar(G::kKFull + x), 1);
+            mbar_init(bar(G::kKEmpty + x), 1);
+        }
+        for (int x = 0; x < G::kNV; ++x) {
+            mbar_init(bar(G::kVFull + x), 1);
+            mbar_init(bar(G::kVEmpty + x), 1);
+        }
+        for (int x = 0; x < 3; ++x) {
+            mbar_init(bar(G::kSFull + x), 1);
+            mbar_init(bar(G::kPFull + x), kGroupWarps);
+            mbar_init(bar(G::kPVDone + x), 1);
+        }
+        for (int x = 0; x < 8; ++x) {
+            mbar_init(bar(G::kMReady + x), 1);     // the publishing warp of the lane quarter
+            mbar_init(bar(G::kLReady + x), 2);     // one warp of each group
+        }
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -253,97 +264,93 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     } else if (warp == kWarpQK || warp == kWarpV) {
         // ------------------------------------------------------------ TMA producers
-        // Stage s of step t is free once the MMA of step t - 2 has completed:
-        // S (the K ring) commits to s_full[t % 3], PV (the V ring) to pv_done[t % 3].
+        // Pair stage x of ring R holds pairs x, x + R, x + 2R, ... (numbered over
+        // the CTA's whole run); pair n may load once the MMA chain of pair n - R
+        // has committed its release (k_empty / v_empty).  A TMA instruction holds
+        // its issuing thread for a long time and one thread's copies complete
+        // roughly one after another, so each box of a pair is issued by its own
+        // lane, all in one instruction.
         const bool kprod = warp == kWarpQK;
-        if (lane == 0) {
-            int n = 0, q_it = 0, it = 0;
-            bool ok = true;
-            const int bFull = kprod ? G::kKFull : G::kVFull;
-            const uint32_t sX = kprod ? sK : sV;
-            while (ok) {
-                const int lb = n & 1;
-                if (!mbar_wait(bar(G::kListFull + lb), (n >> 1) & 1, wc)) {
-                    ok = false;
-                    break;
-                }
-                const TileInfo inf = infos[lb];
-                if (inf.count < 0)
-                    break;
-                const uint16_t *lst = lists + lb * lstride;
-                const int zkv = inf.b * p.Hkv + inf.h / p.g;
-                if (inf.count > 0) {
-                    if (kprod) {
-                        const int qb = q_it & 1;
-                        if (q_it >= 2 && !mbar_wait(bar(G::kQEmpty + qb), ((q_it >> 1) - 1) & 1, wc)) {
-                            ok = false;
-                            break;
-                        }
-                        mbar_arrive_expect_tx(bar(G::kQFull + qb), (uint32_t)G::kQBytes);
-#pragma unroll
-                        for (int pn = 0; pn < G::kPanels; ++pn)
-                            tma_load_3d(sQ + qb * G::kQBytes + pn * 8192, &tmQ, bar(G::kQFull + qb), pn * 64,
-                                        inf.i * 64, inf.b * p.Hq + inf.h);
-                        ++q_it;
-                    }
-                    const int steps = (inf.count + 1) >> 1;
-                    for (int s = 0; s < steps; ++s) {
-                        const int st = it & 1;
-                        const bool freed =
-                            it < 2 || mbar_wait(bar((kprod ? G::kSFull : G::kPVDone) + (it - 2) % 3),
-                                                (uint32_t)(((it - 2) / 3) & 1), wc);
-                        if (!freed) {
-                            ok = false;
-                            break;
-                        }
-                        const int nblk = (2 * s + 1 < inf.count) ? 2 : 1;
-                        mbar_arrive_expect_tx(bar(bFull + st), (uint32_t)(nblk * G::kBlkBytes));
-                        for (int c = 0; c < nblk; ++c) {
-                            const int j = lst[2 * s + c];
-                            if (kprod) {
-                                // [panel][128 keys]: block c fills rows 64c..64c+63 of every panel.
-#pragma unroll
-                                for (int pn = 0; pn < G::kPanels; ++pn)
-                                    tma_load_3d(sX + st * G::kStage + pn * 16384 + c * 8192, &tmK, bar(bFull + st),
-                                                pn * 64, j * 64, zkv);
-                            } else {
-                                // [block][panel][64 keys]: one 4-D box per block.
-                                tma_load_4d(sX + st * G::kStage + c * G::kBlkBytes, &tmV, bar(bFull + st), 0, j * 64,
-                                            0, zkv);
-                            }
-                            const int ta = 2 * s + c + kPrefetchAhead;
-                            if (ta < inf.count) {
-                                const int jp = lst[ta];
-                                if (kprod) {
-#pragma unroll
-                                    for (int pn = 0; pn < G::kPanels; ++pn)
-                                        tma_prefetch_3d(&tmK, pn * 64, jp * 64, zkv);
-                                } else {
-                                    tma_prefetch_4d(&tmV, 0, jp * 64, 0, zkv);
-                                }
-                            }
-                        }
-                        ++it;
-                    }
-                    if (!ok)
-                        break;
-                }
-                mbar_arrive(bar(G::kListEmpty + lb));
-                ++n;
+        const int R = kprod ? G::kNK : G::kNV;
+        int n = 0, q_it = 0, pr = 0;
+        bool ok = true;
+        const int bFull = kprod ? G::kKFull : G::kVFull;
+        const int bEmpty = kprod ? G::kKEmpty : G::kVEmpty;
+        const uint32_t sX = kprod ? sK : sV;
+        while (ok) {
+            const int lb = n & 1;
+            if (!warp_wait(bar(G::kListFull + lb), (n >> 1) & 1, wc)) {
+                ok = false;
+                break;
             }
-            if (!ok) {
-                // Drain the copies this thread issued before the CTA exits.
-                for (int st = 0; st < 2; ++st) {
-                    const int last = ((it - 1) & 1) == st ? it - 1 : it - 2;
-                    if (last >= 0)
-                        mbar_drain(bar(bFull + st), (uint32_t)((last >> 1) & 1), kDrain);
-                }
+            const TileInfo inf = infos[lb];
+            if (inf.count < 0)
+                break;
+            const uint16_t *lst = lists + lb * lstride;
+            const int zkv = inf.b * p.Hkv + inf.h / p.g;
+            if (inf.count > 0) {
                 if (kprod) {
-                    for (int qb = 0; qb < 2; ++qb) {
-                        const int last = ((q_it - 1) & 1) == qb ? q_it - 1 : q_it - 2;
-                        if (last >= 0)
-                            mbar_drain(bar(G::kQFull + qb), (uint32_t)((last >> 1) & 1), kDrain);
+                    const int qb = q_it % G::kQBufs;
+                    if (q_it >= G::kQBufs && !warp_wait(bar(G::kQEmpty + qb), (uint32_t)((q_it / G::kQBufs - 1) & 1), wc)) {
+                        ok = false;
+                        break;
                     }
+                    if (lane == 0)
+                        mbar_arrive_expect_tx(bar(G::kQFull + qb), (uint32_t)G::kQBytes);
+                    __syncwarp();
+                    if (lane < G::kPanels)
+                        tma_load_3d(sQ + qb * G::kQBytes + lane * 8192, &tmQ, bar(G::kQFull + qb), lane * 64,
+                                    inf.i * 64, inf.b * p.Hq + inf.h);
+                    ++q_it;
+                }
+                const int npairs = (inf.count + 1) >> 1;
+                for (int e2 = 0; e2 < npairs; ++e2, ++pr) {
+                    const int st = pr % R;
+                    if (pr >= R && !warp_wait(bar(bEmpty + st), (uint32_t)((pr / R - 1) & 1), wc)) {
+                        ok = false;
+                        break;
+                    }
+                    const int nblk = min(2, inf.count - 2 * e2);
+                    if (lane == 0)
+                        mbar_arrive_expect_tx(bar(bFull + st), (uint32_t)(nblk * G::kBlkBytes));
+                    __syncwarp();
+                    if (kprod) {
+                        // [panel][128 keys]: block c fills rows 64c..64c+63 of every panel.
+                        if (lane < nblk * G::kPanels) {
+                            const int c = lane / G::kPanels, pn = lane % G::kPanels;
+                            tma_load_3d(sX + st * G::kPair + pn * 16384 + c * 8192, &tmK, bar(bFull + st), pn * 64,
+                                        lst[2 * e2 + c] * 64, zkv);
+                        }
+                    } else if (lane < nblk) {
+                        // [block][panel][64 keys]: one 4-D box per block.
+                        tma_load_4d(sX + st * G::kPair + lane * G::kBlkBytes, &tmV, bar(bFull + st), 0,
+                                    lst[2 * e2 + lane] * 64, 0, zkv);
+                    }
+                }
+                if (!ok)
+                    break;
+            }
+            __syncwarp();
+            if (lane == 0)
+                mbar_arrive(bar(G::kListEmpty + lb));
+            ++n;
+        }
+        if (!ok && lane == 0) {
+            // Drain the copies this warp issued before the CTA exits.
+            for (int st = 0; st < R; ++st) {
+                int last = pr - 1;
+                while (last >= 0 && last % R != st)
+                    --last;
+                if (last >= 0)
+                    mbar_drain(bar(bFull + st), (uint32_t)((last / R) & 1), kDrain);
+            }
+            if (kprod) {
+                for (int qb = 0; qb < G::kQBufs; ++qb) {
+                    int last = q_it - 1;
+                    while (last >= 0 && last % G::kQBufs != qb)
+                        --last;
+                    if (last >= 0)
+                        mbar_drain(bar(G::kQFull + qb), (uint32_t)((last / G::kQBufs) & 1), kDrain);
                 }
             }
         }
@@ -355,7 +362,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             // Descriptors advance by (byte offset >> 4) in their start-address field.
             const uint64_t dq0 = smem_desc_sw128(sQ, 16, 1024);
             const uint64_t dk0 = smem_desc_sw128(sK, 16, 1024);
-            int n = 0, q_it = 0, g = 0;
+            int n = 0, q_it = 0, g = 0, pr = 0;
             bool ok = true, issued = false;
             while (ok) {
                 const int lb = n & 1;
@@ -370,25 +377,25 @@ __global__ void __launch_bounds__(kThreads, 1)
                     break;
                 if (count == 0)
                     continue;
-                const int qb = q_it & 1;
-                if (!mbar_wait(bar(G::kQFull + qb), (uint32_t)((q_it >> 1) & 1), wc)) {
+                const int qb = q_it % G::kQBufs;
+                if (!mbar_wait(bar(G::kQFull + qb), (uint32_t)((q_it / G::kQBufs) & 1), wc)) {
                     ok = false;
                     break;
                 }
                 const uint64_t dq = dq0 + (uint64_t)((qb * G::kQBytes) >> 4);
                 const int steps = (count + 1) >> 1;
-                for (int s = 0; s < steps; ++s, ++g) {
-                    const int sb = g & 1;
+                for (int s = 0; s < steps; ++s, ++g, ++pr) {
+                    const int st = pr % G::kNK;
                     // K of this step landed; S buffer g % 3 free: PV(g - 3) has read the P
                     // written over it (and so the softmax has read S(g - 3)).
-                    if (!mbar_wait(bar(G::kKFull + sb), (uint32_t)((g >> 1) & 1), wc) ||
+                    if (!mbar_wait(bar(G::kKFull + st), (uint32_t)((pr / G::kNK) & 1), wc) ||
                         (g >= 3 && !mbar_wait(bar(G::kPVDone + g % 3), (uint32_t)(((g - 3) / 3) & 1), wc))) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
                     const uint32_t id = (2 * s + 1 < count) ? idS2 : idS1;
-                    const uint64_t dk = dk0 + (uint64_t)((sb * G::kStage) >> 4);
+                    const uint64_t dk = dk0 + (uint64_t)((st * G::kPair) >> 4);
 #pragma unroll
                     for (int kk = 0; kk < D / 16; ++kk) {
                         const uint32_t qo = ((kk >> 2) * 8192 + (kk & 3) * 32) >> 4;
@@ -396,6 +403,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         mma_ss(tS(g % 3), dq + qo, dk + ko, id, kk > 0 ? 1u : 0u);
                     }
                     issued = true;
+                    tc_commit(bar(G::kKEmpty + st));
                     tc_commit(bar(G::kSFull + g % 3));
                     if (s == steps - 1)
                         tc_commit(bar(G::kQEmpty + qb));
@@ -414,7 +422,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0) {
             constexpr uint32_t idPV = idesc_bf16(64, D, 1);
             const uint64_t dv0 = smem_desc_sw128(sV, 8192, 1024);
-            int n = 0, o_it = 0, g = 0;
+            int n = 0, o_it = 0, g = 0, pr = 0;
             bool ok = true, issued = false;
             while (ok) {
                 const int lb = n & 1;
@@ -430,25 +438,27 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (count == 0)
                     continue;
                 const int steps = (count + 1) >> 1;
-                for (int s = 0; s < steps; ++s, ++g) {
-                    const int sb = g & 1;
+                for (int s = 0; s < steps; ++s, ++g, ++pr) {
+                    const int st = pr % G::kNV;
                     // The first PV of a tile overwrites O: the previous tile's O must
                     // have been read out (o_free).
                     if (!mbar_wait(bar(G::kPFull + g % 3), (uint32_t)((g / 3) & 1), wc) ||
-                        !mbar_wait(bar(G::kVFull + sb), (uint32_t)((g >> 1) & 1), wc) ||
-                        (s == 0 && o_it >= 1 && !mbar_wait(bar(G::kOFree + (o_it - 1) % 2), (uint32_t)(((o_it - 1) >> 1) & 1), wc))) {
+                        !mbar_wait(bar(G::kVFull + st), (uint32_t)((pr / G::kNV) & 1), wc) ||
+                        (s == 0 && o_it >= 1 &&
+                         !mbar_wait(bar(G::kOFree + ((o_it - 1) & 1)), (uint32_t)(((o_it - 1) >> 1) & 1), wc))) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
                     const int ksteps = (2 * s + 1 < count) ? 8 : 4;
-                    const uint64_t dv = dv0 + (uint64_t)((sb * G::kStage) >> 4);
+                    const uint64_t dv = dv0 + (uint64_t)((st * G::kPair) >> 4);
                     for (int kk = 0; kk < ksteps; ++kk) {
                         // V stage [block][panel][64 keys]: 16 keys per K step, LBO = next d panel.
                         const uint32_t vo = ((kk >> 2) * G::kBlkBytes + (kk & 3) * 2048) >> 4;
-                        mma_ts(tO, tS(g % 3) + kk * 8, dv + vo, idPV, (s == 0 && kk == 0) ? 0u : 1u);
+                        mma_ts(tO, tS(g % 3) + 8u * kk, dv + vo, idPV, (s == 0 && kk == 0) ? 0u : 1u);
                     }
                     issued = true;
+                    tc_commit(bar(G::kVEmpty + st));
                     tc_commit(bar(G::kPVDone + g % 3));
                     if (s == steps - 1)
                         tc_commit(bar(G::kOFull + (o_it & 1)));
@@ -462,48 +472,61 @@ __global__ void __launch_bounds__(kThreads, 1)
                 mbar_drain(bar(G::kDrain + 1), 0, kDrain);
             }
         }
-    } else if (warp < kSoftmaxWarps) {
+    } else if (warp < 2 * kGroupWarps) {
         // ------------------------------------------------------------ softmax + epilogue
+        const int grp = warp >> 2;               // steps of parity grp are this group's
         const int qt = warp & 3;                 // TMEM lane quarter: rows 16 qt .. 16 qt + 15
-        const int hf = warp >> 2;                // which 32 keys of each block this warp exponentiates; half of d
         const int r = qt * 16 + (lane & 15);     // query row of the tile
-        const int c = lane >> 4;                 // key block of the step this thread loads; quarter of d
+        const int c = lane >> 4;                 // key block of the step this thread holds; half of d
         const uint32_t lane_off = (uint32_t)(qt * 32) << 16;
-        const int pair_bar = 1 + qt;             // named barrier of the two warps sharing these rows
-        float *xch = reinterpret_cast<float *>(smem + G::kOffXch);
+        float *mrow = reinterpret_cast<float *>(smem + G::kOffM);      // [step % 2][row]
+        float *lrow = reinterpret_cast<float *>(smem + G::kOffL);      // [tile % 2][group][l, m][row]
         const float sl2 = p.scale_log2;
         int n = 0, o_it = 0, g = 0;
         bool ok = true;
-        // Exchange one float per row (lanes 0..15) with the other warp of the pair;
-        // slots alternate so a slot is only rewritten after the partner has read it.
-        int xcnt = 0;
-        auto pair_xchg = [&](float val) -> float {
-            float *xs = xch + (xcnt & 1) * 128 + qt * 32;
-            if (lane < 16)
-                xs[hf * 16 + lane] = val;
-            pair_bar_sync(pair_bar);
-            const float o = xs[(hf ^ 1) * 16 + (lane & 15)];
-            ++xcnt;
-            return o;
+        // This group's row sum of a tile (both threads of the row), against the
+        // running max m_used of its latest step, handed to the epilogue through
+        // l_ready.
+        auto publish_l = [&](int slot, float l, float m_used) {
+            float *dst = lrow + (slot * 2 + grp) * 2 * 64;
+            l += __shfl_xor_sync(0xffffffffu, l, 16);   // the row's two threads (key blocks 0 and 1)
+            if (lane < 16) {
+                dst[r] = l;
+                dst[64 + r] = m_used;
+            }
+            __syncwarp();
+            if (lane == 0)
+                mbar_arrive(bar(G::kLReady + slot * 4 + qt));
         };
-        // A finished tile whose O is still to be written out.
+        // A finished tile whose O this group reads out (it takes the next step).
         bool pend = false;
-        int pb = 0, ph = 0, pi = 0, po_it = 0;
-        float pm = 0.f, pl = 0.f;
+        int pb = 0, ph = 0, pi = 0, po_it = 0, pg = 0;
+        float pm = 0.f;
         // O -> bf16 -> global (and LSE) for the pending tile, then release O.
         auto epilogue = [&]() -> bool {
+            const int slot = po_it & 1;
+            if (!warp_wait(bar(G::kLReady + slot * 4 + qt), (uint32_t)((po_it >> 1) & 1), wc))
+                return false;
+            float pl = 0.f;
+#pragma unroll
+            for (int x = 0; x < 2; ++x) {
+                const float lx = lrow[(slot * 2 + x) * 2 * 64 + r];
+                const float mx = lrow[(slot * 2 + x) * 2 * 64 + 64 + r];
+                if (lx > 0.f)
+                    pl += lx * ex2_approx(mx - pm);
+            }
             if (!warp_wait(bar(G::kOFull + (po_it & 1)), (uint32_t)((po_it >> 1) & 1), wc))
                 return false;
             tc_fence_after();
             const bool row_ok = pi * 64 + r < p.S;   // rows past S (ragged last block) are never stored
             const size_t orow = (size_t)(pb * p.Hq + ph) * p.S + (size_t)pi * 64 + r;
-            uint4 *dst = reinterpret_cast<uint4 *>(p.o + orow * D + hf * (D / 2) + c * (D / 4));
+            uint4 *dst = reinterpret_cast<uint4 *>(p.o + orow * D + c * (D / 2));
             const float inv_l = pl > 0.f ? 1.0f / pl : 0.f;
-            uint32_t ov[D / 4];
+            uint32_t ov[D / 2];
             if constexpr (D == 128)
-                tmem_ld16x2_32<D / 4>(tO + lane_off + hf * (D / 2), ov);
+                tmem_ld16x2_64<D / 2>(tO + lane_off, ov);
             else
-                tmem_ld16x2_16<D / 4>(tO + lane_off + hf * (D / 2), ov);
+                tmem_ld16x2_32<D / 2>(tO + lane_off, ov);
             tmem_wait_ld();
             tc_fence_before();
             __syncwarp();
@@ -511,7 +534,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 mbar_arrive(bar(G::kOFree + (po_it & 1)));
             if (row_ok) {
 #pragma unroll
-                for (int x = 0; x < D / 32; ++x) {
+                for (int x = 0; x < D / 16; ++x) {
                     uint32_t w[4];
 #pragma unroll
                     for (int k = 0; k < 4; ++k)
@@ -519,7 +542,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                                            __uint_as_float(ov[8 * x + 2 * k + 1]) * inv_l);
                     dst[x] = make_uint4(w[0], w[1], w[2], w[3]);
                 }
-                if (p.lse != nullptr && hf == 0 && c == 0)
+                if (p.lse != nullptr && c == 0)
                     p.lse[orow] = pl > 0.f ? (pm + __log2f(pl)) * 0.69314718055994530942f : -INFINITY;
             }
             pend = false;
@@ -540,159 +563,157 @@ __global__ void __launch_bounds__(kThreads, 1)
                 break;
             const int count = inf.count;
             if (count == 0) {
-                // No selected block: O = 0, LSE = -inf.
-                if (inf.i * 64 + r < p.S) {
+                // No selected block: O = 0, LSE = -inf (written by group 0).
+                if (grp == 0 && inf.i * 64 + r < p.S) {
                     const size_t orow = (size_t)(inf.b * p.Hq + inf.h) * p.S + (size_t)inf.i * 64 + r;
-                    uint4 *dst = reinterpret_cast<uint4 *>(p.o + orow * D + hf * (D / 2) + c * (D / 4));
+                    uint4 *dst = reinterpret_cast<uint4 *>(p.o + orow * D + c * (D / 2));
 #pragma unroll
-                    for (int x = 0; x < D / 32; ++x)
+                    for (int x = 0; x < D / 16; ++x)
                         dst[x] = make_uint4(0u, 0u, 0u, 0u);
-                    if (p.lse != nullptr && hf == 0 && c == 0)
+                    if (p.lse != nullptr && c == 0)
                         p.lse[orow] = -INFINITY;
                 }
                 continue;
             }
             const int diag = inf.diag;
             const int steps = (count + 1) >> 1;
-            float m = -INFINITY, l = 0.f;
-            int s = 0;
-            // One step: S (both key blocks of the row, so the row max is exact in
-            // every warp) -> this warp's 32 keys of each block -> P.  The last step
-            // of a tile (absent second block, diagonal block) is a separate
+            const int g0 = g;
+            float l = 0.f, m_used = -INFINITY;
+            // One step (global number g, step s of the tile): this thread's 64 scores
+            // -> row max -> running max (handed on) -> exponentials -> P.  The last
+            // step of a tile (absent second block, diagonal block) is a separate
             // instantiation so the other steps carry no masking code.
-            auto step = [&](auto last_c) -> bool {
+            auto step = [&](auto last_c, int s) -> bool {
                 constexpr bool kLast = decltype(last_c)::value;
-                if (!warp_wait(bar(G::kSFull + g % 3), (uint32_t)((g / 3) & 1), wc))
+                const int b = g % 3;
+                if (!warp_wait(bar(G::kSFull + b), (uint32_t)((g / 3) & 1), wc))
                     return false;
                 tc_fence_after();
-                // Thread c holds key block c: v = this warp's 32 keys (32 hf ..), w = the
-                // other warp's 32 (only their max is needed).
-                const int e = 2 * s + c;              // list entry of this thread's key block
-                const uint32_t tSg = tS(g % 3);
-                uint32_t v[32], w[32];
-                tmem_ld16x2_32<64>(tSg + lane_off + hf * 32, v);
-                tmem_ld16x2_32<64>(tSg + lane_off + (hf ^ 1) * 32, w);
+                uint32_t v[64];
+                tmem_ld16x2_64<64>(tS(b) + lane_off, v);
                 tmem_wait_ld();
                 if constexpr (kLast) {
-                    // Keys kept in each half: none for an absent block; up to the query
-                    // row in the diagonal block (causal); all otherwise.
-                    const bool dg = diag && e == count - 1;
-                    const int lim_v = e >= count ? 0 : dg ? min(max(r - 32 * hf + 1, 0), 32) : 32;
-                    const int lim_w = e >= count ? 0 : dg ? min(max(r - 32 * (hf ^ 1) + 1, 0), 32) : 32;
+                    // Keys kept: none for an absent block; up to the query row in the
+                    // diagonal block (causal); all otherwise.
+                    const int e = 2 * s + c;              // list entry of this thread's key block
+                    const int lim = e >= count ? 0 : (diag && e == count - 1) ? r + 1 : 64;
 #pragma unroll
-                    for (int k = 0; k < 32; ++k) {
-                        v[k] = k < lim_v ? v[k] : 0xFF800000u;
-                        w[k] = k < lim_w ? w[k] : 0xFF800000u;
-                    }
+                    for (int k = 0; k < 64; ++k)
+                        v[k] = k < lim ? v[k] : 0xFF800000u;
                 }
-                // Exponentials against the current max m while the exact row max is
-                // formed; both warps of the pair see the same row, so they take the
-                // same decision.  The step is redone when the max grew by more than
-                // 2^8 (and always on a tile's first step, where m is not set yet).
                 float mx8[8];
 #pragma unroll
                 for (int k = 0; k < 8; ++k)
-                    mx8[k] = __uint_as_float(w[k]);
+                    mx8[k] = __uint_as_float(v[k]);
 #pragma unroll
-                for (int k = 8; k < 32; ++k)
-                    mx8[k & 7] = fmaxf(mx8[k & 7], __uint_as_float(w[k]));
-                float ls[4] = {0.f, 0.f, 0.f, 0.f};
-                uint32_t pk[16];
-                {
-                    const float neg_m = -m;
-#pragma unroll
-                    for (int k = 0; k < 16; ++k) {
-                        const float p0 = ex2_approx(fmaf(__uint_as_float(v[2 * k]), sl2, neg_m));
-                        const float p1 = ex2_approx(fmaf(__uint_as_float(v[2 * k + 1]), sl2, neg_m));
-                        ls[k & 3] += p0 + p1;
-                        pk[k] = pack_bf16x2(p0, p1);
-                        mx8[(2 * k) & 7] = fmaxf(mx8[(2 * k) & 7], __uint_as_float(v[2 * k]));
-                        mx8[(2 * k + 1) & 7] = fmaxf(mx8[(2 * k + 1) & 7], __uint_as_float(v[2 * k + 1]));
-                    }
-                }
+                for (int k = 8; k < 64; ++k)
+                    mx8[k & 7] = fmaxf(mx8[k & 7], __uint_as_float(v[k]));
                 float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
                                  fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
                 mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16)) * sl2;
-                const bool grow = mx > m + 8.0f;
-                if (__any_sync(0xffffffffu, grow)) {
-                    const float m_new = grow ? mx : m;
-                    const bool need = grow && (m != -INFINITY);
-                    if (__any_sync(0xffffffffu, need)) {
-                        // O holds PV up to step g - 1 of this tile: rescale this thread's d columns.
-                        const float alpha = need ? ex2_approx(m - m_new) : 1.0f;
-                        l *= alpha;
-                        if (!warp_wait(bar(G::kPVDone + (g - 1) % 3), (uint32_t)(((g - 1) / 3) & 1), wc))
-                            return false;
-                        tc_fence_after();
-#pragma unroll 1
-                        for (int ch = 0; ch < D / 64; ++ch) {
-                            uint32_t ov[16];
-                            tmem_ld16x2_16<D / 4>(tO + lane_off + hf * (D / 2) + ch * 16, ov);
-                            tmem_wait_ld();
+                // Running max after step g - 1 (the other group's).  At a tile's first
+                // step it is the previous tile's final max, kept for that tile's epilogue.
+                float m_prev = -INFINITY;
+                if (g >= 1) {
+                    const int ps = (g - 1) & 1;
+                    if (!warp_wait(bar(G::kMReady + ps * 4 + qt), (uint32_t)(((g - 1) >> 1) & 1), wc))
+                        return false;
+                    const float mp = mrow[ps * 64 + r];
+                    if (s == 0)
+                        pm = mp;
+                    else
+                        m_prev = mp;
+                }
+                const float m_new = mx > m_prev + 8.0f ? mx : m_prev;
+                if (lane < 16)
+                    mrow[(g & 1) * 64 + r] = m_new;
+                __syncwarp();
+                if (lane == 0)
+                    mbar_arrive(bar(G::kMReady + (g & 1) * 4 + qt));
+                if (m_new != m_used) {
+                    l = m_used == -INFINITY ? 0.f : l * ex2_approx(m_used - m_new);
+                    m_used = m_new;
+                }
+                float ls[4] = {0.f, 0.f, 0.f, 0.f};
+                uint32_t pk[32];
+                const float neg_m = -m_new;
 #pragma unroll
-                            for (int k = 0; k < 16; ++k)
-                                ov[k] = __float_as_uint(__uint_as_float(ov[k]) * alpha);
-                            tmem_st16x2_16<D / 4>(tO + lane_off + hf * (D / 2) + ch * 16, ov);
-                        }
-                    }
-                    m = m_new;
-                    const float neg_m = -m;
-#pragma unroll
-                    for (int k = 0; k < 4; ++k)
-                        ls[k] = 0.f;
-#pragma unroll
-                    for (int k = 0; k < 16; ++k) {
-                        const float p0 = ex2_approx(fmaf(__uint_as_float(v[2 * k]), sl2, neg_m));
-                        const float p1 = ex2_approx(fmaf(__uint_as_float(v[2 * k + 1]), sl2, neg_m));
-                        ls[k & 3] += p0 + p1;
-                        pk[k] = pack_bf16x2(p0, p1);
-                    }
+                for (int k = 0; k < 32; ++k) {
+                    const float p0 = ex2_approx(fmaf(__uint_as_float(v[2 * k]), sl2, neg_m));
+                    const float p1 = ex2_approx(fmaf(__uint_as_float(v[2 * k + 1]), sl2, neg_m));
+                    ls[k & 3] += p0 + p1;
+                    pk[k] = pack_bf16x2(p0, p1);
                 }
                 l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
-                // Both warps of the pair have loaded S(g): P may overwrite it.  Keys
-                // 32 hf + 2k, +1 of block c go to column 32 c + 16 hf + k.
-                tc_fence_before();
-                pair_bar_sync(pair_bar);
-                tc_fence_after();
-                tmem_st16x2_16<32>(tSg + lane_off + hf * 16, pk);
+                // O holds this tile's PV up to step g - 1 against m_prev: rescale this
+                // thread's half of d when the max moved.
+                const bool need = s > 0 && m_new != m_prev;
+                if (__any_sync(0xffffffffu, need)) {
+                    const float alpha = need ? ex2_approx(m_prev - m_new) : 1.0f;
+                    if (!warp_wait(bar(G::kPVDone + (g - 1) % 3), (uint32_t)(((g - 1) / 3) & 1), wc))
+                        return false;
+                    tc_fence_after();
+#pragma unroll 1
+                    for (int ch = 0; ch < D / 32; ++ch) {
+                        uint32_t ov[16];
+                        tmem_ld16x2_16<D / 2>(tO + lane_off + ch * 16, ov);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int k = 0; k < 16; ++k)
+                            ov[k] = __float_as_uint(__uint_as_float(ov[k]) * alpha);
+                        tmem_st16x2_16<D / 2>(tO + lane_off + ch * 16, ov);
+                    }
+                    tmem_wait_st();
+                }
+                // P over the first 64 columns of this S buffer: only this warp reads
+                // these lanes of it, and its loads have completed.  Keys 2k, 2k + 1
+                // of block c go to column 32 c + k.
+                tmem_st16x2_32<32>(tS(b) + lane_off, pk);
                 tmem_wait_st();
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0)
-                    mbar_arrive(bar(G::kPFull + g % 3));
+                    mbar_arrive(bar(G::kPFull + b));
                 // The previous tile's O: its last PV finished while this step ran;
                 // this tile's first PV waits for it to be read out.
                 if (pend && !epilogue())
                     return false;
                 return true;
             };
-            for (; s < steps; ++s, ++g) {
-                const bool good = (s + 1 < steps) ? step(std::false_type{}) : step(std::true_type{});
+            int s = (g0 & 1) == grp ? 0 : 1;
+            if (s >= steps)
+                publish_l(o_it & 1, 0.f, -INFINITY);   // a one-step tile of the other group
+            for (; s < steps; s += 2) {
+                g = g0 + s;
+                const bool good = (s + 1 < steps) ? step(std::false_type{}, s) : step(std::true_type{}, s);
                 if (!good) {
                     ok = false;
                     break;
                 }
+                if (s + 2 >= steps)
+                    publish_l(o_it & 1, l, m_used);
             }
             if (!ok)
                 break;
-            // Row sum over the four threads that hold the row (two per warp).
-            l += __shfl_xor_sync(0xffffffffu, l, 16);
-            pl = l + pair_xchg(l);
-            pend = true;
-            pb = inf.b;
-            ph = inf.h;
-            pi = inf.i;
-            po_it = o_it;
-            pm = m;
+            g = g0 + steps;
+            // The group that takes the next step reads this tile's O out.
+            if ((g & 1) == grp) {
+                pend = true;
+                pb = inf.b;
+                ph = inf.h;
+                pi = inf.i;
+                po_it = o_it;
+                pg = g - 1;
+            }
             ++o_it;
         }
-        if (ok && pend)
-            epilogue();
-        if (!ok) {
-            // The partner warp may be waiting at a pair barrier (at most two come
-            // between bounded waits, which see the abort flag): release it.
-            pair_bar_arrive(pair_bar);
-            pair_bar_arrive(pair_bar);
+        if (ok && pend) {
+            // No further step: take the pending tile's final max, then read O out.
+            const int ps = pg & 1;
+            if (warp_wait(bar(G::kMReady + ps * 4 + qt), (uint32_t)((pg >> 1) & 1), wc)) {
+                pm = mrow[ps * 64 + r];
+                epilogue();
+            }
         }
     }
 
