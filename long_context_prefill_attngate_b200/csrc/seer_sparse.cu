@@ -35,8 +35,9 @@
 //    A tcgen05.mma issue blocks at the tensor pipe's rate and every commit or
 //    barrier check of the issuing thread is serial latency; with two issuers
 //    one thread's checks are covered by the other's MMAs.
-//  * K and V rings of pair stages (two key blocks each); each MMA chain commits
-//    the release of the stage it read.  A TMA instruction holds its issuing
+//  * K and V rings of two stages (one step's two key blocks each): a stage is
+//    free once the S (or PV) MMA of the step two back has completed, which the
+//    s_full (pv_done) commit already signals.  A TMA instruction holds its issuing
 //    thread for a long time and one thread's copies complete roughly one after
 //    another, so every box of a stage is issued by its own lane.
 //  * Warps: 0-7 softmax and epilogue (a tile's O -> bf16 -> global and LSE are
@@ -58,12 +59,6 @@
 #include "seer_internal.h"
 #include "seer_ptx.cuh"
 
-#ifndef SEER_NK
-#define SEER_NK 2
-#endif
-#ifndef SEER_NV
-#define SEER_NV 2
-#endif
 
 namespace seer {
 
@@ -100,7 +95,7 @@ struct Geo {
     static constexpr int kQBytes = 64 * D * 2;        // one query block
     static constexpr int kBlkBytes = 64 * D * 2;      // one key block (K or V)
     static constexpr int kPair = 2 * kBlkBytes;       // a stage: two key blocks
-    static constexpr int kNK = SEER_NK, kNV = SEER_NV; // ring depths in stages
+    static constexpr int kNK = 2, kNV = 2;            // ring depths in stages (step n reuses step n - 2's)
     static constexpr int kQBufs = 2;                  // query-block buffers
     static constexpr int kOffK = kQBufs * kQBytes;
     static constexpr int kOffV = kOffK + kNK * kPair;
@@ -111,8 +106,7 @@ struct Geo {
     // m_ready[slot][quarter] hands the running max from one softmax group to the
     // other (slot = step % 2); l_ready[slot][quarter] collects both groups' row
     // sums of a tile (slot = tile % 2).
-    static constexpr int kQFull = 0, kQEmpty = 2, kKFull = 4, kKEmpty = kKFull + kNK, kVFull = kKEmpty + kNK,
-                         kVEmpty = kVFull + kNV, kSFull = kVEmpty + kNV, kPFull = kSFull + 3, kPVDone = kPFull + 3,
+    static constexpr int kQFull = 0, kQEmpty = 2, kKFull = 4, kVFull = kKFull + kNK, kSFull = kVFull + kNV, kPFull = kSFull + 3, kPVDone = kPFull + 3,
                          kOFull = kPVDone + 3, kOFree = kOFull + 2, kListFull = kOFree + 2, kListEmpty = kListFull + 2,
                          kDrain = kListEmpty + 2, kMReady = kDrain + 2, kLReady = kMReady + 8, kNumBars = kLReady + 8;
     static constexpr int kOffM = kOffBar + kNumBars * 8;           // float [2 slots][64 rows]
@@ -163,14 +157,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(bar(G::kListEmpty + x), kListConsumers);
             mbar_init(bar(G::kDrain + x), 1);
         }
-        for (int x = 0; x < G::kNK; ++x) {
+        for (int x = 0; x < G::kNK; ++x)
             mbar_init(bar(G::kKFull + x), 1);
-            mbar_init(bar(G::kKEmpty + x), 1);
-        }
-        for (int x = 0; x < G::kNV; ++x) {
+        for (int x = 0; x < G::kNV; ++x)
             mbar_init(bar(G::kVFull + x), 1);
-            mbar_init(bar(G::kVEmpty + x), 1);
-        }
         for (int x = 0; x < 3; ++x) {
             mbar_init(bar(G::kSFull + x), 1);
             mbar_init(bar(G::kPFull + x), kGroupWarps);
@@ -264,9 +254,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     } else if (warp == kWarpQK || warp == kWarpV) {
         // ------------------------------------------------------------ TMA producers
-        // Pair stage x of ring R holds pairs x, x + R, x + 2R, ... (numbered over
-        // the CTA's whole run); pair n may load once the MMA chain of pair n - R
-        // has committed its release (k_empty / v_empty).  A TMA instruction holds
+        // One stage per step; stage x of a ring of two holds steps x, x + 2, ...
+        // (numbered over the CTA's whole run).  Step n may load once the MMA that
+        // read step n - 2 has completed: S(n - 2) (s_full) for K, PV(n - 2)
+        // (pv_done) for V, both kept per step % 3.  A TMA instruction holds
         // its issuing thread for a long time and one thread's copies complete
         // roughly one after another, so each box of a pair is issued by its own
         // lane, all in one instruction.
@@ -275,7 +266,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         int n = 0, q_it = 0, pr = 0;
         bool ok = true;
         const int bFull = kprod ? G::kKFull : G::kVFull;
-        const int bEmpty = kprod ? G::kKEmpty : G::kVEmpty;
+        const int bDone = kprod ? G::kSFull : G::kPVDone;
         const uint32_t sX = kprod ? sK : sV;
         while (ok) {
             const int lb = n & 1;
@@ -306,7 +297,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int npairs = (inf.count + 1) >> 1;
                 for (int e2 = 0; e2 < npairs; ++e2, ++pr) {
                     const int st = pr % R;
-                    if (pr >= R && !warp_wait(bar(bEmpty + st), (uint32_t)((pr / R - 1) & 1), wc)) {
+                    if (pr >= R && !warp_wait(bar(bDone + (pr - R) % 3), (uint32_t)(((pr - R) / 3) & 1), wc)) {
                         ok = false;
                         break;
                     }
@@ -403,7 +394,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                         mma_ss(tS(g % 3), dq + qo, dk + ko, id, kk > 0 ? 1u : 0u);
                     }
                     issued = true;
-                    tc_commit(bar(G::kKEmpty + st));
                     tc_commit(bar(G::kSFull + g % 3));
                     if (s == steps - 1)
                         tc_commit(bar(G::kQEmpty + qb));
@@ -450,15 +440,21 @@ __global__ void __launch_bounds__(kThreads, 1)
                         break;
                     }
                     tc_fence_after();
-                    const int ksteps = (2 * s + 1 < count) ? 8 : 4;
                     const uint64_t dv = dv0 + (uint64_t)((st * G::kPair) >> 4);
-                    for (int kk = 0; kk < ksteps; ++kk) {
-                        // V stage [block][panel][64 keys]: 16 keys per K step, LBO = next d panel.
-                        const uint32_t vo = ((kk >> 2) * G::kBlkBytes + (kk & 3) * 2048) >> 4;
-                        mma_ts(tO, tS(g % 3) + 8u * kk, dv + vo, idPV, (s == 0 && kk == 0) ? 0u : 1u);
-                    }
+                    const uint32_t tp = tS(g % 3);
+                    // V stage [block][panel][64 keys]: 16 keys per K step, LBO = next d panel.
+                    auto chain = [&](auto nk) {
+#pragma unroll
+                        for (int kk = 0; kk < decltype(nk)::value; ++kk) {
+                            const uint32_t vo = ((kk >> 2) * G::kBlkBytes + (kk & 3) * 2048) >> 4;
+                            mma_ts(tO, tp + 8u * kk, dv + vo, idPV, (s == 0 && kk == 0) ? 0u : 1u);
+                        }
+                    };
+                    if (2 * s + 1 < count)
+                        chain(std::integral_constant<int, 8>{});
+                    else
+                        chain(std::integral_constant<int, 4>{});
                     issued = true;
-                    tc_commit(bar(G::kVEmpty + st));
                     tc_commit(bar(G::kPVDone + g % 3));
                     if (s == steps - 1)
                         tc_commit(bar(G::kOFull + (o_it & 1)));
