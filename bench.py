@@ -517,7 +517,7 @@ def run_gpu(args, world, rank, local):
         "config": {"workload": w_full.name, "B": w_full.B, "Hq": w_full.Hq, "Hkv": w_full.Hkv, "S": w_full.S,
                    "d": w_full.d, "mask": "gate-topk", "density_target": args.density,
                    "density": round(density_meas, 4), "d_gate": w_full.d_gate, "rope_theta": w_full.rope_theta,
-                   "l2": "flushed between timed steps (256 MiB write, outside the step events)",
+                   "l2": "flushed between timed GPU steps (256 MiB write, outside the step events); the host oracle arm has no GPU cache",
                    "parallelism": ("single" if world == 1 else
                                    f"kv-head split x{world}" if args.split == "heads" else f"replicas x{world}")},
         "ms_layer_attention": round(ms_attn, 4), "ms_gate": round(ms_gate, 4), "ms_mask": round(ms_mask, 4),
@@ -773,7 +773,7 @@ def run_reference(args, world, rank):
                       "mask": "gate-topk", "density_target": args.density,
                       "density": round(float(mask.sum()) / (w.B * w.Hq * w.nb * (w.nb + 1) / 2), 4),
                       "d_gate": w.d_gate, "rope_theta": w.rope_theta,
-                      "l2": "host oracle: no GPU cache to flush",
+                      "l2": "flushed between timed GPU steps (256 MiB write, outside the step events); the host oracle arm has no GPU cache",
                       "parallelism": "single"},
            "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample},
            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
