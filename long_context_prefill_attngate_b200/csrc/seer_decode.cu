@@ -451,10 +451,17 @@ __global__ void __launch_bounds__(D)
 #pragma unroll
     for (int w = 0; w < D / 32; ++w)
         lt += sred[1][w];
+    // Every split's value of dim t first (all loads in flight together), then the
+    // weighted sum in split order.
+    float vals[kMaxDecodeSplits];
+#pragma unroll
+    for (int s2 = 0; s2 < kMaxDecodeSplits; ++s2)
+        vals[s2] = s2 < nsplit ? pp[s2 * (D + 2) + t] : 0.f;
     float acc = 0.f;
-#pragma unroll 8
-    for (int s2 = 0; s2 < nsplit; ++s2)
-        acc = fmaf(sw[s2], pp[s2 * (D + 2) + t], acc);
+#pragma unroll
+    for (int s2 = 0; s2 < kMaxDecodeSplits; ++s2)
+        if (s2 < nsplit)
+            acc = fmaf(sw[s2], vals[s2], acc);
     const bool has = lt > 0.f;
     o[bh * D + t] = __float2bfloat16(has ? acc / lt : 0.f);
     if (lse != nullptr && t == 0)
