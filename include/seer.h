@@ -196,6 +196,11 @@ SEER_API seer_status seer_compact_mask(const seer_shape *shape, const uint8_t *m
  * device error that seer_check_status reports as SEER_ERR_DEVICE.  A CUDA
  * graph that captured the call reuses its counter on every replay, so one
  * graph must not be replayed on two streams at once.
+ * Shared memory: the kernel's layout grows with nb (two key-block lists of nb
+ * entries); at d = 128 and the largest nb it leaves under 1 KB of the 227 KB
+ * window for aligning the window's base to 1 KB.  The kernel checks that its
+ * aligned layout fits before it touches shared memory; if not it writes
+ * nothing and records a device error (SEER_ERR_DEVICE from seer_check_status).
  */
 SEER_API seer_status seer_block_sparse_prefill(const seer_shape *shape, const void *q, const void *k,
                                       const void *v, const uint8_t *mask, float softmax_scale,

@@ -468,6 +468,9 @@ seer_status seer_check_status(void *stream)
         if (v == kStatusRing)
             return fail(SEER_ERR_DEVICE, "more than 256 attention launches were in flight at once: a tile-counter "
                                          "slot was reused by a later launch (outputs of the earlier one are incomplete)");
+        if (v == kStatusSmem)
+            return fail(SEER_ERR_DEVICE, "the attention kernel's shared-memory layout did not fit its window once "
+                                         "aligned (no output was written)");
         return fail(SEER_ERR_DEVICE, "device-side check failed (code %d)", v);
     }
     return ok();

@@ -9,8 +9,9 @@
 namespace seer {
 
 // Device status codes written through the status pointer every kernel gets
-// (first error wins).
-enum : int { kStatusOk = 0, kStatusTimeout = 5, kStatusDevice = 6, kStatusRing = 7 };
+// (first error wins).  kStatusSmem: a kernel found its shared-memory layout,
+// after aligning the window's base, larger than the dynamic window it was given.
+enum : int { kStatusOk = 0, kStatusTimeout = 5, kStatusDevice = 6, kStatusRing = 7, kStatusSmem = 8 };
 
 __device__ __forceinline__ void set_status(int *status, int s)
 {

@@ -115,7 +115,11 @@ struct Geo {
     static constexpr int kOffMisc = kOffInfo + 2 * (int)sizeof(TileInfo);
     static constexpr int kOffList = (kOffMisc + 16 + 15) / 16 * 16;
     static int list_stride(int nb) { return (nb + 7) / 8 * 8; }    // uint16 entries per buffer
-    static int smem_bytes(int nb) { return kOffList + 2 * list_stride(nb) * 2 + 1024; }
+    // Bytes the layout uses from its 1024-aligned base; the window asked for adds up
+    // to 1 KB for aligning the base, as much of it as the 227 KB cap leaves (the
+    // kernel checks that the aligned layout fits the window it got).
+    static int smem_used(int nb) { return kOffList + 2 * list_stride(nb) * 2; }
+    static int smem_bytes(int nb) { return smem_used(nb) + 1024 < 227 * 1024 ? smem_used(nb) + 1024 : 227 * 1024; }
 };
 
 __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, const WaitCtx &w)
@@ -147,6 +151,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     const WaitCtx wc{abort_flag, p.timeout_ns, p.status};
     const int lstride = p.list_stride;
 
+    {   // the aligned layout must fit the dynamic window (uniform over the grid)
+        uint32_t window;
+        asm volatile("mov.u32 %0, %%dynamic_smem_size;" : "=r"(window));
+        const uint32_t pad = (uint32_t)(reinterpret_cast<uintptr_t>(smem) - reinterpret_cast<uintptr_t>(smem_raw));
+        if (pad + (uint32_t)G::kOffList + 4u * (uint32_t)lstride > window) {
+            if (threadIdx.x == 0)
+                set_status(p.status, kStatusSmem);
+            return;
+        }
+    }
     if (threadIdx.x == 0) {
         for (int x = 0; x < 2; ++x) {
             mbar_init(bar(G::kQFull + x), 1);
@@ -747,7 +761,7 @@ cudaError_t launch_d(const AttnLaunch &a, cudaStream_t stream)
     p.tile_base = a.tile_base;
     p.list_stride = Geo<D>::list_stride(a.nb);
     const int smem = Geo<D>::smem_bytes(a.nb);
-    if (smem > 227 * 1024)
+    if (Geo<D>::smem_used(a.nb) > 227 * 1024)
         return cudaErrorInvalidValue;
     auto kern = sparse_attn_kernel<D>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);

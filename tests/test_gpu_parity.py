@@ -277,9 +277,12 @@ def test_prefill_concurrent_streams_and_counter_ring():
     assert torch.equal(o, ref2)
 
 
-def test_prefill_max_sequence(oracle):
-    """S = 2^20 (the largest nb the library accepts): first + diagonal blocks only."""
-    B, Hq, Hkv, S, d = 1, 2, 1, 1 << 20, 64
+@pytest.mark.parametrize("d", [64, 128])
+def test_prefill_max_sequence(oracle, d):
+    """S = 2^20 (the largest nb the library accepts): first + diagonal blocks only.
+    At d = 128 the kernel's shared-memory layout leaves almost no room under the
+    227 KB cap, so this also covers the window-fit check passing."""
+    B, Hq, Hkv, S = 1, 2, 1, 1 << 20
     nb = S // BLOCK
     g = torch.Generator().manual_seed(77)
     q = torch.randn((B, Hq, S, d), generator=g).to(torch.bfloat16)
@@ -287,6 +290,14 @@ def test_prefill_max_sequence(oracle):
     v = torch.randn((B, Hkv, S, d), generator=g).to(torch.bfloat16)
     scores = torch.zeros((B, Hq, nb, nb), dtype=torch.float32, device="cuda")
     mask = seer.seer_block_mask(scores, "topk", k_fixed=2, Hkv=Hkv, d=d)
+    for _, h, i in [(0, h, i) for h in range(Hq) for i in (0, 1, 5000, nb - 1)]:
+        row = mask[0, h, i].cpu().numpy()
+        want = np.zeros(nb, np.uint8)
+        want[0] = 1
+        want[i] = 1
+        assert np.array_equal(row, want)
+    if d == 128:
+        mask[0, 0, nb - 1].fill_(1)    # one full row: a 16384-entry key-block list
     o = seer.seer_block_sparse_prefill(dev(q), dev(k), dev(v), mask)
     seer.seer_check_status()
     units = np.array([(0, h, i) for h in range(Hq) for i in (0, 1, 5000, nb - 1)], np.int32)
@@ -296,13 +307,7 @@ def test_prefill_max_sequence(oracle):
     for _, h, i in units:
         mask_rows[0, h, i] = mask[0, h, i].cpu()
     o_ref, _ = oracle.masked_attention(bits(q), bits(k), bits(v), mask_rows.numpy(), units=units)
-    check_o(gather_units(o.cpu(), units), o_ref, "O@1M")
-    for _, h, i in units:
-        row = mask[0, h, i].cpu().numpy()
-        want = np.zeros(nb, np.uint8)
-        want[0] = 1
-        want[i] = 1
-        assert np.array_equal(row, want)
+    check_o(gather_units(o.cpu(), units), o_ref, f"O@1M d={d}")
 
 
 # ------------------------------------------------------------------ pooled map
