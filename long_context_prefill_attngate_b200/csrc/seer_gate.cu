@@ -9,11 +9,15 @@
 //  Question 2 — the soft scores of a row sum to 1.
 //
 // Three kernels, all fp32 arithmetic:
-//  1. pool_kernel:        Q and K read once with 16-byte loads (HBM-bound);
-//  2. project_rope_kernel: per-head d x d_gate projection + block RoPE;
-//  3. gate_softmax_kernel: causal block logits Qt_i . Kt_j / sqrt(d_gate)
-//                          and the row softmax over j <= i.
+//  1. pool_kernel:           Q and K read once with 16-byte loads (HBM-bound);
+//  2. project_rope_t_kernel: per-head d x d_gate projection + block RoPE,
+//                            stored feature-major (project_rope_kernel: the
+//                            same rows block-major, for the decode gate);
+//  3. gate_softmax_t_kernel: causal block logits Qt_i . Kt_j / sqrt(d_gate)
+//                            and the row softmax over j <= i.
 #include <cuda_bf16.h>
+
+#include <algorithm>
 
 #include "seer_internal.h"
 
@@ -270,171 +274,399 @@ __global__ void __launch_bounds__(kProjThreads)
     }
 }
 
-constexpr int kLR = 32;              // query blocks per CTA (16, 64, 128 measured slower)
-constexpr int kLThreads = 256;       // 16 x 16: rows ty + 16a, columns tx + 16b
-constexpr int kLTy = kLThreads / 16; // thread rows
-constexpr int kLA = kLR / kLTy;      // query rows per thread
-constexpr int kLC = 64;              // key blocks per tile
-constexpr int kLPad = 4;             // row padding (floats): conflict-free float4 reads
+// ---------------------------------------------------------------- prefill gate
+// The prefill gate keeps its projected rows transposed, [B*H, dg, nb] (feature
+// major), so that the logits kernel reads both operands as contiguous runs of
+// blocks.
 
-// Causal block logits + row softmax for kLR query blocks of one head.  Each
-// thread computes kLA x 4 logits per kLR x 64 tile from float4 reads of the
-// shared Qt and Kt rows; raw logits (times 1/sqrt(dg)) go to `scores` while
-// each row's running max and exp-sum are kept online (the 16 threads sharing
-// a row reduce with shuffles).  A second pass over the same tiles writes
-// exp(x - m) / sum, and the entries j > i are set to 0.
-constexpr int kLPF = 8;              // float4 per thread of a prefetched Kt tile (d_gate <= 128)
+__device__ __forceinline__ void cpa16(uint32_t dst, const void *src)
+{
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cpa_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cpa_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 
-template <bool PF>
-__global__ void __launch_bounds__(kLThreads)
-    gate_softmax_kernel(const float *__restrict__ qt, const float *__restrict__ kt, int Hq, int Hkv, int nb, int dg,
-                        float scale, float *__restrict__ scores)
+constexpr int kPTR = 64;               // rows per pass: 8 per warp
+constexpr int kPTThreads = 256;
+
+struct ProjTJob {
+    const float *xp;                   // pooled rows [nbh, nb, d]
+    int H, d, nbh;                     // heads of the weights, input features, B * H
+    const __nv_bfloat16 *w;            // [H] x (d x dg), w_stride apart
+    long long w_stride;
+    float *out;                        // [nbh, dg, nb]
+};
+
+// Both projections of the prefill gate in one persistent launch.  The rows of
+// the two jobs, in groups of 8 ("octets", head-major), are split over the grid
+// in proportion to their cost (d FMAs per output), so every CTA has the same
+// work whatever the head counts; a CTA takes its range in passes of up to 64
+// rows of one head and reloads W only when the head changes.  Warp w owns rows
+// 8w .. 8w + 7 of a pass and lane l the rotation pairs (t, t + dg/2) for
+// t = 2l, 2l + 1 (+ 64 per further column pass): x is read from shared memory
+// as two broadcast float4 (rows of one feature are contiguous) and W as two
+// bf16 pairs, for 16 packed FMAs on row pairs.  Each output is the fmaf chain
+// over the features in order, as in project_rope_kernel; RoPE angles as there.
+__global__ void __launch_bounds__(kPTThreads, 2)
+    project_rope_t_kernel(const ProjTJob j0, const ProjTJob j1, int nb, int dg, double theta)
+{
+    extern __shared__ float4 ptsm4[];
+    const int dmax = max(j0.d, j1.d);
+    float *sx = reinterpret_cast<float *>(ptsm4);                              // [d][kPTR]
+    uint32_t *sw = reinterpret_cast<uint32_t *>(sx + (size_t)dmax * kPTR);     // bf16 pairs [d][dg / 2]
+    double *sfreq = reinterpret_cast<double *>(sw + (size_t)dmax * dg / 2);
+    const int half = dg / 2;
+    for (int t = threadIdx.x; t < half; t += kPTThreads)
+        sfreq[t] = pow(theta, -2.0 * (double)t / (double)dg);
+    const int noh = (nb + 7) / 8;                                               // octets per head
+    const long long n0 = (long long)j0.nbh * noh, n1 = (long long)j1.nbh * noh;
+    const long long c0 = n0 * j0.d, ctot = c0 + n1 * j1.d;
+    // first octet whose cumulative cost reaches `target`
+    auto oct_at = [&](long long target) -> long long {
+        return target <= c0 ? (target + j0.d - 1) / j0.d : n0 + (target - c0 + j1.d - 1) / j1.d;
+    };
+    const long long ob = oct_at(ctot * blockIdx.x / gridDim.x);
+    const long long oe = oct_at(ctot * (blockIdx.x + 1) / gridDim.x);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    constexpr double kTwoPi = 6.283185307179586476925286766559;
+    int cur_job = -1, cur_h = -1;
+    for (long long o = ob; o < oe;) {
+        const int jb = o < n0 ? 0 : 1;
+        const ProjTJob &job = jb ? j1 : j0;
+        const long long lo = o - (jb ? n0 : 0);
+        const int bh = (int)(lo / noh), oi = (int)(lo % noh);
+        const long long job_end = jb ? n0 + n1 : n0;
+        const int noct = (int)min(min(oe, job_end) - o, (long long)min(8, noh - oi));
+        const int i0 = oi * 8, rows = min(8 * noct, nb - i0);
+        const int d = job.d, h = bh % job.H;
+        __syncthreads();                                   // the previous pass is done with sx / sw
+        if (jb != cur_job || h != cur_h) {
+            const __nv_bfloat16 *wh = job.w + (long long)h * job.w_stride;
+            const int words = d * dg / 2;
+            if ((reinterpret_cast<uintptr_t>(wh) & 15) == 0 && (words & 3) == 0) {
+                const uint4 *w4 = reinterpret_cast<const uint4 *>(wh);
+                for (int e = threadIdx.x; e < words / 4; e += kPTThreads)
+                    reinterpret_cast<uint4 *>(sw)[e] = __ldg(w4 + e);
+            } else {
+                const unsigned short *w16 = reinterpret_cast<const unsigned short *>(wh);
+                for (int e = threadIdx.x; e < words; e += kPTThreads)
+                    sw[e] = (uint32_t)w16[2 * e] | ((uint32_t)w16[2 * e + 1] << 16);
+            }
+            cur_job = jb;
+            cur_h = h;
+        }
+        // x transposed: thread e takes 8 features (32 bytes) of row e % 64
+        for (int e = threadIdx.x; e < kPTR * (d / 8); e += kPTThreads) {
+            const int r = e & (kPTR - 1), c8 = e / kPTR;
+            float4 a = make_float4(0.f, 0.f, 0.f, 0.f), b = a;
+            if (r < rows) {
+                const float4 *src = reinterpret_cast<const float4 *>(job.xp + ((long long)bh * nb + i0 + r) * d + 8 * c8);
+                a = src[0];
+                b = src[1];
+            }
+            float *dst = sx + 8 * c8 * kPTR + r;
+            dst[0 * kPTR] = a.x;
+            dst[1 * kPTR] = a.y;
+            dst[2 * kPTR] = a.z;
+            dst[3 * kPTR] = a.w;
+            dst[4 * kPTR] = b.x;
+            dst[5 * kPTR] = b.y;
+            dst[6 * kPTR] = b.z;
+            dst[7 * kPTR] = b.w;
+        }
+        __syncthreads();
+        if (8 * warp < rows) {
+            const int hw = dg / 2;                                          // W words per feature
+            for (int t0 = 0; t0 < half; t0 += 64) {
+                const int t = t0 + 2 * lane;
+                const bool tok = t < half;                                  // half is even: t + 1 < half too
+                const int wa_i = tok ? t / 2 : 0, wb_i = tok ? (t + half) / 2 : 0;
+                // acc2[p][x]: rows (2p, 2p + 1) of output column x, two packed fmaf chains
+                float2 acc2[4][4];
+#pragma unroll
+                for (int p2 = 0; p2 < 4; ++p2)
+#pragma unroll
+                    for (int x = 0; x < 4; ++x)
+                        acc2[p2][x] = make_float2(0.f, 0.f);
+                const float *xr = sx + 8 * warp;
+#pragma unroll 4
+                for (int c = 0; c < d; ++c) {
+                    const float4 xa = *reinterpret_cast<const float4 *>(xr + c * kPTR);
+                    const float4 xb = *reinterpret_cast<const float4 *>(xr + c * kPTR + 4);
+                    const uint32_t wa = sw[c * hw + wa_i], wb = sw[c * hw + wb_i];
+                    const float wv[4] = {__uint_as_float(wa << 16), __uint_as_float(wa & 0xffff0000u),
+                                         __uint_as_float(wb << 16), __uint_as_float(wb & 0xffff0000u)};
+                    const float2 xp2[4] = {make_float2(xa.x, xa.y), make_float2(xa.z, xa.w), make_float2(xb.x, xb.y),
+                                           make_float2(xb.z, xb.w)};
+#pragma unroll
+                    for (int x = 0; x < 4; ++x) {
+                        const float2 w2 = make_float2(wv[x], wv[x]);
+#pragma unroll
+                        for (int p2 = 0; p2 < 4; ++p2)
+                            acc2[p2][x] = fma2(xp2[p2], w2, acc2[p2][x]);
+                    }
+                }
+                float acc[8][4];
+#pragma unroll
+                for (int p2 = 0; p2 < 4; ++p2)
+#pragma unroll
+                    for (int x = 0; x < 4; ++x) {
+                        acc[2 * p2][x] = acc2[p2][x].x;
+                        acc[2 * p2 + 1][x] = acc2[p2][x].y;
+                    }
+                if (!tok)
+                    continue;
+                // RoPE: column pair (t + q, t + q + half) of row i
+#pragma unroll
+                for (int k = 0; k < 8; ++k) {
+                    const int i = i0 + 8 * warp + k;
+#pragma unroll
+                    for (int q = 0; q < 2; ++q) {
+                        const double ang = (double)i * sfreq[t + q];
+                        const double red = ang - rint(ang * (1.0 / kTwoPi)) * kTwoPi;
+                        float sn, cs;
+                        sincosf((float)red, &sn, &cs);
+                        const float v0 = acc[k][q], v1 = acc[k][2 + q];
+                        acc[k][q] = v0 * cs - v1 * sn;
+                        acc[k][2 + q] = v1 * cs + v0 * sn;
+                    }
+                }
+                const int cols[4] = {t, t + 1, t + half, t + half + 1};
+                const int r0 = 8 * warp;
+                if ((nb & 3) == 0 && r0 + 8 <= rows) {
+#pragma unroll
+                    for (int x = 0; x < 4; ++x) {
+                        float4 *dst = reinterpret_cast<float4 *>(job.out + ((long long)bh * dg + cols[x]) * nb + i0 + r0);
+                        dst[0] = make_float4(acc[0][x], acc[1][x], acc[2][x], acc[3][x]);
+                        dst[1] = make_float4(acc[4][x], acc[5][x], acc[6][x], acc[7][x]);
+                    }
+                } else {
+#pragma unroll
+                    for (int x = 0; x < 4; ++x)
+#pragma unroll
+                        for (int k = 0; k < 8; ++k)
+                            if (r0 + k < rows)
+                                job.out[((long long)bh * dg + cols[x]) * nb + i0 + r0 + k] = acc[k][x];
+                }
+            }
+        }
+        o += noct;
+    }
+}
+
+constexpr int kSR = 64;                // query blocks per CTA: 8 per warp
+constexpr int kSC = 128;               // key blocks per tile: 4 per lane
+constexpr int kSK = 64;                // features per pipeline stage
+constexpr int kSThreads = 256;
+
+// Causal block logits Qt_i . Kt_j / sqrt(dg) and the row softmax over j <= i
+// for 64 query blocks of one head, from the transposed rows.  Warp w owns
+// rows 8w .. 8w + 7 and lane l the columns 4l .. 4l + 3 of a 128-column tile:
+// per feature two broadcast float4 of Qt and one float4 of Kt feed 16 packed
+// FMAs on row pairs.  Kt arrives in (tile, 64-feature) stages through a
+// two-deep cp.async ring.  Each tile's raw logits are stored; a second pass by
+// the same threads reads them back for the row's max and exp-sum (per lane,
+// then across the warp) and writes exp(x - m) / sum, and 0 for j > i up to nb.  CTA order: the first `split` CTAs take the heaviest chunks
+// of every head, the rest the remaining chunks lightest first, so that CTAs
+// sharing an SM even out.
+__global__ void __launch_bounds__(kSThreads, 2)
+    gate_softmax_t_kernel(const float *__restrict__ qt, const float *__restrict__ kt, int Hq, int Hkv, int nbh,
+                          int nb, int dg, float scale, int split, float *__restrict__ scores)
 {
     extern __shared__ float4 gsm4[];
-    const int rs = dg + kLPad;
-    float *sq = reinterpret_cast<float *>(gsm4);           // kLR x rs
-    float *sk = sq + kLR * rs;                             // kLC x rs
-    const int bh = blockIdx.x;                             // b * Hq + h
+    float *sq = reinterpret_cast<float *>(gsm4);          // [dg][kSR]
+    float *sk = sq + (size_t)dg * kSR;                    // [2][kSK][kSC]
+    const int nchunk = (nb + kSR - 1) / kSR;
+    const int total = nbh * nchunk;
+    const int u = blockIdx.x;
+    const int rank = u < split ? u : split + (total - 1 - u);
+    const int bh = rank % nbh, chunk = nchunk - 1 - rank / nbh;
     const int b = bh / Hq, h = bh % Hq;
-    const int g = Hq / Hkv;
-    // Heaviest query chunks (most causal columns) of every head first.
-    const int i0 = (gridDim.y - 1 - blockIdx.y) * kLR;
-    const int rows = min(kLR, nb - i0);
-    const float *qbase = qt + ((long long)bh * nb + i0) * dg;
-    const float *kbase = kt + ((long long)(b * Hkv + h / g) * nb) * dg;
-    const int dg4 = dg / 4;
-    for (int e = threadIdx.x; e < kLR * dg4; e += kLThreads) {
-        const int r = e / dg4, c4 = e % dg4;
-        const float4 v = r < rows ? reinterpret_cast<const float4 *>(qbase + (long long)r * dg)[c4]
-                                  : make_float4(0.f, 0.f, 0.f, 0.f);
-        *reinterpret_cast<float4 *>(sq + r * rs + 4 * c4) = v;
-    }
-    const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
-    const int jlast = i0 + rows - 1;
-    float m[kLA], ssum[kLA];
-#pragma unroll
-    for (int a = 0; a < kLA; ++a) {
-        m[a] = -INFINITY;
-        ssum[a] = 0.f;
-    }
-    // PF: the next Kt tile is loaded into registers while this one is used,
-    // hiding the L2 latency of the tile loads.
-    float4 pf[PF ? kLPF : 1];
-    auto fetch = [&](int jt) {
-        const int nc = min(kLC, jlast + 1 - jt);
-#pragma unroll
-        for (int it = 0; it < kLPF; ++it) {
-            const int e = threadIdx.x + it * kLThreads;
-            const int jj = e / dg4, c4 = e % dg4;
-            pf[it] = (e < kLC * dg4 && jj < nc) ? reinterpret_cast<const float4 *>(kbase + (long long)(jt + jj) * dg)[c4]
-                                                : make_float4(0.f, 0.f, 0.f, 0.f);
+    const int hk = b * Hkv + h / (Hq / Hkv);
+    const int i0 = chunk * kSR, rows = min(kSR, nb - i0);
+    const int jend = i0 + rows;                           // columns [0, jend)
+    const int ntile = (jend + kSC - 1) / kSC, nkc = (dg + kSK - 1) / kSK, nsteps = ntile * nkc;
+    const float *qsrc = qt + (size_t)bh * dg * nb;
+    const float *ksrc = kt + (size_t)hk * dg * nb;
+    const bool vec = (nb & 3) == 0;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int r0 = 8 * warp;
+    const bool wrows = r0 < rows;                         // this warp has rows
+    const int imax = i0 + min(r0 + 8, rows) - 1;          // its last row
+
+    // Qt rows i0 .. i0 + 63 of every feature
+    if (vec) {
+        for (int e = threadIdx.x; e < dg * (kSR / 4); e += kSThreads) {
+            const int c = e / (kSR / 4), x = e % (kSR / 4);
+            float *dst = sq + c * kSR + 4 * x;
+            if (4 * x < rows)
+                cpa16(static_cast<uint32_t>(__cvta_generic_to_shared(dst)), qsrc + (size_t)c * nb + i0 + 4 * x);
+            else
+                *reinterpret_cast<float4 *>(dst) = make_float4(0.f, 0.f, 0.f, 0.f);
         }
-    };
-    if (PF)
-        fetch(0);
-    for (int j0 = 0; j0 <= jlast; j0 += kLC) {
-        __syncthreads();
-        if (PF) {
-#pragma unroll
-            for (int it = 0; it < kLPF; ++it) {
-                const int e = threadIdx.x + it * kLThreads;
-                if (e < kLC * dg4)
-                    *reinterpret_cast<float4 *>(sk + (e / dg4) * rs + 4 * (e % dg4)) = pf[it];
+    } else {
+        for (int e = threadIdx.x; e < dg * kSR; e += kSThreads) {
+            const int c = e / kSR, r = e % kSR;
+            sq[e] = r < rows ? qsrc[(size_t)c * nb + i0 + r] : 0.f;
+        }
+    }
+    auto load_stage = [&](int s) {
+        const int tile = s / nkc, kc = s % nkc;
+        const int j0 = tile * kSC, c0 = kc * kSK, nc = min(kSK, dg - c0);
+        float *dst0 = sk + (size_t)(s & 1) * kSK * kSC;
+        if (vec) {
+            for (int e = threadIdx.x; e < nc * (kSC / 4); e += kSThreads) {
+                const int c = e / (kSC / 4), x = e % (kSC / 4);
+                float *dst = dst0 + c * kSC + 4 * x;
+                if (j0 + 4 * x < jend)
+                    cpa16(static_cast<uint32_t>(__cvta_generic_to_shared(dst)), ksrc + (size_t)(c0 + c) * nb + j0 + 4 * x);
+                else
+                    *reinterpret_cast<float4 *>(dst) = make_float4(0.f, 0.f, 0.f, 0.f);
             }
         } else {
-            const int ncols = min(kLC, jlast + 1 - j0);
-            for (int e = threadIdx.x; e < kLC * dg4; e += kLThreads) {
-                const int jj = e / dg4, c4 = e % dg4;
-                const float4 v = jj < ncols ? reinterpret_cast<const float4 *>(kbase + (long long)(j0 + jj) * dg)[c4]
-                                            : make_float4(0.f, 0.f, 0.f, 0.f);
-                *reinterpret_cast<float4 *>(sk + jj * rs + 4 * c4) = v;
+            for (int e = threadIdx.x; e < nc * kSC; e += kSThreads) {
+                const int c = e / kSC, x = e % kSC;
+                dst0[c * kSC + x] = j0 + x < jend ? ksrc[(size_t)(c0 + c) * nb + j0 + x] : 0.f;
             }
         }
+    };
+    load_stage(0);
+    cpa_commit();
+
+    float2 acc2[4][4];                                    // rows (2p, 2p + 1) of column 4 lane + x
+    for (int s = 0; s < nsteps; ++s) {
+        if (s + 1 < nsteps)
+            load_stage(s + 1);                            // its buffer was released at the end of step s - 1
+        cpa_commit();
+        cpa_wait<1>();
         __syncthreads();
-        if (PF && j0 + kLC <= jlast)
-            fetch(j0 + kLC);
-        float acc[kLA][4];
+        const int tile = s / nkc, kc = s % nkc;
+        const int j0 = tile * kSC;
+        const bool live = wrows && j0 <= imax;            // the warp has a row reaching this tile
+        if (kc == 0) {
 #pragma unroll
-        for (int a = 0; a < kLA; ++a)
+            for (int p2 = 0; p2 < 4; ++p2)
 #pragma unroll
-            for (int c = 0; c < 4; ++c)
-                acc[a][c] = 0.f;
-#pragma unroll 1
-        for (int c = 0; c < dg; c += 4) {
-            float4 qv[kLA], kv[4];
-#pragma unroll
-            for (int a = 0; a < kLA; ++a)
-                qv[a] = *reinterpret_cast<const float4 *>(sq + (ty + kLTy * a) * rs + c);
-#pragma unroll
-            for (int bb = 0; bb < 4; ++bb)
-                kv[bb] = *reinterpret_cast<const float4 *>(sk + (tx + 16 * bb) * rs + c);
-#pragma unroll
-            for (int a = 0; a < kLA; ++a)
-#pragma unroll
-                for (int bb = 0; bb < 4; ++bb)
-                    acc[a][bb] = fmaf(qv[a].x, kv[bb].x,
-                                      fmaf(qv[a].y, kv[bb].y, fmaf(qv[a].z, kv[bb].z, fmaf(qv[a].w, kv[bb].w, acc[a][bb]))));
+                for (int x = 0; x < 4; ++x)
+                    acc2[p2][x] = make_float2(0.f, 0.f);
         }
+        if (live) {
+            const int c0 = kc * kSK, nc = min(kSK, dg - c0);
+            const float *qr = sq + (size_t)c0 * kSR + r0;
+            const float *kr = sk + (size_t)(s & 1) * kSK * kSC + 4 * lane;
+#pragma unroll 4
+            for (int c = 0; c < nc; ++c) {
+                const float4 qa = *reinterpret_cast<const float4 *>(qr + c * kSR);
+                const float4 qb = *reinterpret_cast<const float4 *>(qr + c * kSR + 4);
+                const float4 kv = *reinterpret_cast<const float4 *>(kr + c * kSC);
+                const float2 q2[4] = {make_float2(qa.x, qa.y), make_float2(qa.z, qa.w), make_float2(qb.x, qb.y),
+                                      make_float2(qb.z, qb.w)};
+                const float kx[4] = {kv.x, kv.y, kv.z, kv.w};
 #pragma unroll
-        for (int a = 0; a < kLA; ++a) {
-            const int r = ty + kLTy * a;
-            const int i = i0 + r;
+                for (int x = 0; x < 4; ++x) {
+                    const float2 k2 = make_float2(kx[x], kx[x]);
+#pragma unroll
+                    for (int p2 = 0; p2 < 4; ++p2)
+                        acc2[p2][x] = fma2(q2[p2], k2, acc2[p2][x]);
+                }
+            }
+        }
+        if (kc == nkc - 1 && live) {
+            // raw scaled logits of this tile (entries j > i are overwritten in the second pass)
+            const int jl = j0 + 4 * lane;
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+                const int r = r0 + k, i = i0 + r;
+                if (r >= rows)                            // warp-uniform
+                    break;
+                float v[4];
+#pragma unroll
+                for (int x = 0; x < 4; ++x)
+                    v[x] = ((k & 1) ? acc2[k >> 1][x].y : acc2[k >> 1][x].x) * scale;
+                float *row = scores + ((size_t)bh * nb + i) * nb;
+                if (vec) {
+                    if (jl < nb)
+                        *reinterpret_cast<float4 *>(row + jl) = make_float4(v[0], v[1], v[2], v[3]);
+                } else {
+#pragma unroll
+                    for (int x = 0; x < 4; ++x)
+                        if (jl + x < nb)
+                            row[jl + x] = v[x];
+                }
+            }
+        }
+        __syncthreads();                                  // buffer s & 1 is free for step s + 2
+    }
+    cpa_wait<0>();
+    // Second pass over what this thread stored: the row's max and exp-sum (each
+    // lane over its own columns, then combined across the warp), then
+    // exp(x - m) / sum, and 0 for j > i up to nb.
+    if (!wrows)
+        return;
+    for (int k = 0; k < 8; ++k) {
+        const int r = r0 + k, i = i0 + r;
+        if (r >= rows)
+            break;
+        float *row = scores + ((size_t)bh * nb + i) * nb;
+        float mx = -INFINITY, sm = 0.f;
+        for (int jl = 4 * lane; jl <= i; jl += kSC) {
+            float v[4];
+            if (vec) {
+                const float4 f = *reinterpret_cast<const float4 *>(row + jl);
+                v[0] = f.x;
+                v[1] = f.y;
+                v[2] = f.z;
+                v[3] = f.w;
+            } else {
+#pragma unroll
+                for (int x = 0; x < 4; ++x)
+                    v[x] = jl + x <= i ? row[jl + x] : 0.f;
+            }
             float tm = -INFINITY;
 #pragma unroll
-            for (int bb = 0; bb < 4; ++bb) {
-                const int j = j0 + tx + 16 * bb;
-                acc[a][bb] *= scale;
-                if (r < rows && j <= i) {
-                    scores[((long long)bh * nb + i) * nb + j] = acc[a][bb];
-                    tm = fmaxf(tm, acc[a][bb]);
-                }
-            }
-#pragma unroll
-            for (int off = 1; off < 16; off <<= 1)
-                tm = fmaxf(tm, __shfl_xor_sync(0xffffffffu, tm, off));
-            const float mn = fmaxf(m[a], tm);
+            for (int x = 0; x < 4; ++x)
+                if (jl + x <= i)
+                    tm = fmaxf(tm, v[x]);
+            const float mn = fmaxf(mx, tm);
             float ts = 0.f;
 #pragma unroll
-            for (int bb = 0; bb < 4; ++bb) {
-                const int j = j0 + tx + 16 * bb;
-                if (r < rows && j <= i)
-                    ts += expf(acc[a][bb] - mn);
-            }
-#pragma unroll
-            for (int off = 1; off < 16; off <<= 1)
-                ts += __shfl_xor_sync(0xffffffffu, ts, off);
-            if (mn != -INFINITY) {
-                ssum[a] = (m[a] == -INFINITY ? 0.f : ssum[a] * expf(m[a] - mn)) + ts;
-                m[a] = mn;
-            }
+            for (int x = 0; x < 4; ++x)
+                if (jl + x <= i)
+                    ts += expf(v[x] - mn);
+            sm = (mx == -INFINITY ? 0.f : sm * expf(mx - mn)) + ts;
+            mx = mn;
         }
-    }
-    // Normalise: each thread rereads exactly the logits it wrote.
-    for (int j0 = 0; j0 <= jlast; j0 += kLC) {
+        float mt = mx;
 #pragma unroll
-        for (int a = 0; a < kLA; ++a) {
-            const int r = ty + kLTy * a;
-            const int i = i0 + r;
-            if (r >= rows)
-                continue;
-            const float inv = 1.0f / ssum[a];
+        for (int off = 16; off > 0; off >>= 1)
+            mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, off));
+        float lt = mx == -INFINITY ? 0.f : sm * expf(mx - mt);   // lane 0 holds block 0: mt is finite
 #pragma unroll
-            for (int bb = 0; bb < 4; ++bb) {
-                const int j = j0 + tx + 16 * bb;
-                if (j <= i) {
-                    float *p = scores + ((long long)bh * nb + i) * nb + j;
-                    *p = expf(*p - m[a]) * inv;
+        for (int off = 16; off > 0; off >>= 1)
+            lt += __shfl_xor_sync(0xffffffffu, lt, off);
+        const float inv = 1.0f / lt;
+        for (int jl = 4 * lane; jl < nb; jl += kSC) {
+            if (vec) {
+                float v[4] = {0.f, 0.f, 0.f, 0.f};
+                if (jl <= i) {
+                    const float4 f = *reinterpret_cast<const float4 *>(row + jl);
+                    v[0] = f.x;
+                    v[1] = f.y;
+                    v[2] = f.z;
+                    v[3] = f.w;
                 }
+#pragma unroll
+                for (int x = 0; x < 4; ++x)
+                    v[x] = jl + x <= i ? expf(v[x] - mt) * inv : 0.f;
+                *reinterpret_cast<float4 *>(row + jl) = make_float4(v[0], v[1], v[2], v[3]);
+            } else {
+#pragma unroll
+                for (int x = 0; x < 4; ++x)
+                    if (jl + x < nb)
+                        row[jl + x] = jl + x <= i ? expf(row[jl + x] - mt) * inv : 0.f;
             }
         }
-    }
-    // Zeros above the diagonal.
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    for (int r = warp; r < rows; r += kLThreads / 32) {
-        const int i = i0 + r;
-        float *row = scores + ((long long)bh * nb + i) * nb;
-        for (int j = i + 1 + lane; j < nb; j += 32)
-            row[j] = 0.f;
     }
 }
 
@@ -525,6 +757,16 @@ size_t gate_projection_smem(int d_in, int dg)
     return sizeof(float) * (kProjRows * (d_in + kPStride) + (size_t)d_in * dg) + sizeof(double) * (dg / 2) + 16;
 }
 
+size_t gate_projection_t_smem(int d_in, int dg)
+{
+    return sizeof(float) * (size_t)kPTR * d_in + sizeof(uint16_t) * (size_t)d_in * dg + sizeof(double) * (dg / 2);
+}
+
+size_t gate_softmax_t_smem(int dg)
+{
+    return sizeof(float) * ((size_t)dg * kSR + 2 * (size_t)kSK * kSC);
+}
+
 cudaError_t launch_gate(int B, int Hq, int Hkv, int S, int d, int dg, float theta, bool k_maxmin, const void *q,
                         const void *k, const void *wq, long long wq_stride, const void *wk, long long wk_stride,
                         float *scores, void *ws, cudaStream_t stream)
@@ -558,30 +800,41 @@ cudaError_t launch_gate(int B, int Hq, int Hkv, int S, int d, int dg, float thet
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess)
         return e;
-    const size_t psmem = gate_projection_smem(dk, dg);    // dk >= d: covers both jobs
-    e = cudaFuncSetAttribute(project_rope_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)psmem);
+    int dev = 0, sms = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess)
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const size_t psmem = gate_projection_t_smem(dk, dg);  // dk >= d: covers both jobs
+    e = cudaFuncSetAttribute(project_rope_t_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)psmem);
     if (e != cudaSuccess)
         return e;
-    const ProjJob jq{qp, Hq, d, static_cast<const __nv_bfloat16 *>(wq), wq_stride, qt};
-    const ProjJob jk{kp, Hkv, dk, static_cast<const __nv_bfloat16 *>(wk), wk_stride, kt};
-    const dim3 pg(B * (Hq + Hkv), (nb + kProjRows - 1) / kProjRows);
-    project_rope_kernel<<<pg, kProjThreads, psmem, stream>>>(jq, jk, B * Hq, nb, nb, dg, (double)theta, 0);
+    e = cudaFuncSetAttribute(project_rope_t_kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                             cudaSharedmemCarveoutMaxShared);
+    if (e != cudaSuccess)
+        return e;
+    int per_sm = 1;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, project_rope_t_kernel, kPTThreads, psmem);
+    if (e != cudaSuccess)
+        return e;
+    const ProjTJob jq{qp, Hq, d, B * Hq, static_cast<const __nv_bfloat16 *>(wq), wq_stride, qt};
+    const ProjTJob jk{kp, Hkv, dk, B * Hkv, static_cast<const __nv_bfloat16 *>(wk), wk_stride, kt};
+    const long long octs = (long long)B * (Hq + Hkv) * ((nb + 7) / 8);
+    const int pgrid = (int)std::min<long long>(octs, (long long)sms * std::max(per_sm, 1));
+    project_rope_t_kernel<<<pgrid, kPTThreads, psmem, stream>>>(jq, jk, nb, dg, (double)theta);
     e = cudaGetLastError();
     if (e != cudaSuccess)
         return e;
-    const size_t ssmem = sizeof(float) * (size_t)(kLR + kLC) * (dg + kLPad);
-    const bool pf = kLC * (dg / 4) <= kLPF * kLThreads;
-    e = cudaFuncSetAttribute(pf ? gate_softmax_kernel<true> : gate_softmax_kernel<false>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ssmem);
+    const size_t ssmem = gate_softmax_t_smem(dg);
+    e = cudaFuncSetAttribute(gate_softmax_t_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ssmem);
     if (e != cudaSuccess)
         return e;
-    const dim3 sg(B * Hq, (nb + kLR - 1) / kLR);
-    if (pf)
-        gate_softmax_kernel<true><<<sg, kLThreads, ssmem, stream>>>(qt, kt, Hq, Hkv, nb, dg, 1.0f / sqrtf((float)dg),
-                                                                   scores);
-    else
-        gate_softmax_kernel<false><<<sg, kLThreads, ssmem, stream>>>(qt, kt, Hq, Hkv, nb, dg, 1.0f / sqrtf((float)dg),
-                                                                    scores);
+    e = cudaFuncSetAttribute(gate_softmax_t_kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                             cudaSharedmemCarveoutMaxShared);
+    if (e != cudaSuccess)
+        return e;
+    const int nchunk = (nb + kSR - 1) / kSR;
+    const int sgrid = B * Hq * nchunk;
+    gate_softmax_t_kernel<<<sgrid, kSThreads, ssmem, stream>>>(qt, kt, Hq, Hkv, B * Hq, nb, dg,
+                                                               1.0f / sqrtf((float)dg), std::min(sgrid, sms), scores);
     return cudaGetLastError();
 }
 
