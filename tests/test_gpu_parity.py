@@ -342,6 +342,21 @@ def test_gate_scores(oracle, B, Hq, Hkv, S, d, dg):
     check_rel(s.cpu().numpy(), ref, "scores")
 
 
+@pytest.mark.parametrize("B,Hq,Hkv,S,d,dg", [(1, 4, 2, 1000, 128, 256), (2, 3, 3, 700, 64, 12),
+                                             (1, 2, 1, 37 * BLOCK + 5, 128, 4)])
+def test_gate_scores_dgate_range(oracle, B, Hq, Hkv, S, d, dg):
+    """d_gate above one 64-feature stage of the logits kernel (256: four stages,
+    the projection's second column pass), below one warp's rotation pairs
+    (12, 4); block counts 16 (the 16-byte load path), 11 and 38 (not multiples
+    of 4: the element-wise path)."""
+    w = syn.custom("gatedg", B, Hq, Hkv, S, d, number=53 + S + dg, d_gate=dg)
+    x = syn.make_inputs(w)
+    s = seer.seer_gate_scores(dev(x["q"]), dev(x["k"]), dev(x["wq"]), dev(x["wk"]), rope_theta=w.rope_theta)
+    seer.seer_check_status()
+    ref = oracle.gate_scores(bits(x["q"]), bits(x["k"]), bits(x["wq"]), bits(x["wk"]), theta=w.rope_theta)
+    check_rel(s.cpu().numpy(), ref, f"scores(d_gate={dg})")
+
+
 @pytest.mark.parametrize("B,Hq,Hkv,S,d,dg", [(1, 2, 2, 512, 64, 64), (1, 8, 2, 4096, 128, 128),
                                              (2, 5, 1, 1152, 128, 64)])
 def test_gate_scores_maxmin_k(oracle, B, Hq, Hkv, S, d, dg):
