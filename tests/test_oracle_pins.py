@@ -154,8 +154,10 @@ def _np_gate(q, k, wq, wk, theta):
     return e / e.sum(-1, keepdims=True)
 
 
-def test_gate_scores_brute_force(oracle):
-    B, Hq, Hkv, S, d, dg = 1, 4, 2, 512, 32, 16
+@pytest.mark.parametrize("dg", [4, 12, 16])
+def test_gate_scores_brute_force(oracle, dg):
+    """Also at d_gate 4 and 12 (rotation halves of 2 and 6 features)."""
+    B, Hq, Hkv, S, d = 1, 4, 2, 512, 32
     qb, kb = rand_bits((B, Hq, S, d), 12, scale=4.0), rand_bits((B, Hkv, S, d), 13, scale=4.0, shift=0.5)
     wqb, wkb = rand_bits((Hq, d, dg), 14, scale=0.5), rand_bits((Hkv, d, dg), 15, scale=0.5)
     got = oracle.gate_scores(qb, kb, wqb, wkb, theta=1e2)
